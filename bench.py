@@ -1,0 +1,414 @@
+"""Benchmark of the VAR-Q packed-KV hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--bits B] [--impl ours|reference]
+
+One step = plan the cache (host), quantize+pack K and V of the whole cache
+(varq_quantize_pack, two launches), then fused packed-KV attention of the
+query block over every cached token (varq_packed_attention).  Default
+workload: the Infinity-8B-like next-scale 1024px layer (B=2 CFG pair, 32 heads,
+D=128, 13 scales / 10,521 tokens, 4096-token query block), INT4, with INT2
+measured the same way and reported under "also".
+
+Printed (rank 0, one JSON line): the metric, whole-job value (attention
+TFLOP/s over the full step time), per-kernel CUDA-event times, the roofline
+of the dominant kernel (attention, tensor-bound) and of quantize+pack
+(HBM-bound) against the measured peaks in MEASURED_PEAKS.json, the CPU
+oracle timed on a bounded sample (cpu_baseline), the end-to-end number
+through the C ABI with host buffers (e2e), SM clocks sampled during the timed
+region, and the number of library kernel launches.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of
+the workload (the path shards by (batch, head) with no exchange), so scaling
+is weak; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from packed_kv_attention_b200 import synth  # noqa: E402
+
+METRIC = "fused packed-KV attention TFLOP/s and quant+pack GB/s at INT4/INT2 (% of roofline)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def attention_flops(w, lq):
+    return 4.0 * w.batch * w.heads * lq * w.n_tokens * w.head_dim
+
+
+def quant_bytes(L, w):
+    """Algorithmic bytes of one quantize+pack of K and V: bf16 read once,
+    packed words and metadata written once."""
+    bf16 = w.batch * w.heads * w.n_tokens * w.head_dim * 2
+    return 2 * (bf16 + L.packed_bytes + L.meta_bytes)
+
+
+def attention_bytes(L, w, lq, rope):
+    qo = 2 * w.batch * w.heads * lq * w.head_dim * 2
+    kv = 2 * (L.packed_bytes + L.meta_bytes)
+    tables = (w.n_tokens * w.head_dim // 2 * 4 * 2) if rope else 0
+    return qo + kv + tables
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        busy = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- our arm
+
+class Pipeline:
+    """Device buffers and the step of one workload at one bit width."""
+
+    def __init__(self, w, bits, lq, device, seed=0):
+        from packed_kv_attention_b200 import varq as V
+        self.V = V
+        self.w, self.bits, self.lq = w, bits, lq
+        data = synth.make_inputs(w, lq=lq, seed=seed, device=device)
+        self.k, self.v, self.q = data["k"], data["v"], data["q"]
+        self.cos, self.sin = data.get("rope_cos"), data.get("rope_sin")
+        self.bs = data["block_start"]
+        self.L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, self.bs)
+        self.kp, self.km = V.alloc_cache(self.L, device)
+        self.vp, self.vm = V.alloc_cache(self.L, device)
+        self.out = torch.empty_like(self.q)
+        ws = V.varq_packed_attention_workspace(self.L, lq, w.n_blocks)
+        self.ws = torch.empty(max(ws // 4, 1), dtype=torch.float32, device=device)
+        self.launches_per_step = 2 + (1 if ws == 0 else 2)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(self, stream, ev=None):
+        V = self.V
+        self.L = V.varq_cache_alloc(self.w.batch, self.w.heads, self.w.head_dim, self.bits, self.bs)
+        if ev is not None:
+            ev[0].record(stream)
+        V.varq_quantize_pack(self.L, self.k, self.kp, self.km, dev_status=self.status, stream=stream)
+        V.varq_quantize_pack(self.L, self.v, self.vp, self.vm, dev_status=self.status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        V.varq_packed_attention(self.L, self.q, self.kp, self.km, self.vp, self.vm, self.out,
+                                rope_cos=self.cos, rope_sin=self.sin, workspace=self.ws,
+                                dev_status=self.status, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+
+def time_ours(pipe, steps, warmup, stream, dist_ok):
+    for _ in range(warmup):
+        pipe.step(stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_ok:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        pipe.step(stream, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist_ok:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    qp = [e[0].elapsed_time(e[1]) for e in evs]
+    at = [e[1].elapsed_time(e[2]) for e in evs]
+    return total_ms, qp, at
+
+
+def time_e2e(pipe, steps, warmup, stream):
+    """The same step through the C ABI with host buffers: pinned host K, V, Q
+    copied in and the output copied out inside the timed region."""
+    hk = pipe.k.cpu().pin_memory()
+    hv = pipe.v.cpu().pin_memory()
+    hq = pipe.q.cpu().pin_memory()
+    ho = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
+
+    def one():
+        pipe.k.copy_(hk, non_blocking=True)
+        pipe.v.copy_(hv, non_blocking=True)
+        pipe.q.copy_(hq, non_blocking=True)
+        pipe.step(stream)
+        ho.copy_(pipe.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            one()
+        e.record(stream)
+        torch.cuda.synchronize()
+    h2d = (hk.numel() + hv.numel() + hq.numel()) * 2
+    d2h = ho.numel() * 2
+    return s.elapsed_time(e) / steps, h2d, d2h
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, bits, lq, rows, seed=0):
+    """Bounded CPU sample of one step: quantize+pack+dequantize K and V of one
+    (batch, head) slice, then fp64 attention of `rows` query rows over it.
+    Returns (seconds, attention flops of the sample, description)."""
+    from oracle import varq_oracle as O
+    data = synth.make_inputs(w, lq=lq, seed=seed, device="cpu", batch=1, heads=1)
+    bs = data["block_start"]
+    kb = data["k"].view(torch.int16).numpy().view(np.uint16)
+    vb = data["v"].view(torch.int16).numpy().view(np.uint16)
+    qb = data["q"][0, 0].view(torch.int16).numpy().view(np.uint16)
+    rsel = np.arange(min(rows, lq))
+    cos = data.get("rope_cos")
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):  # one host core: numpy's BLAS would otherwise fan out
+        t0 = time.perf_counter()
+        hats = []
+        for xb in (kb, vb):
+            codes, s, mn = O.quantize(xb, bs, bits)
+            words = O.pack(codes, bits)
+            meta = O.meta_words(s, mn)
+            hats.append(O.dequantize(O.unpack(words, bits, bs[-1]), meta, bs)[0, 0])
+        O.attention(qb, hats[0], hats[1], rope_cos=None if cos is None else cos.numpy(),
+                    rope_sin=None if cos is None else data["rope_sin"].numpy(), rows=rsel)
+        dt = time.perf_counter() - t0
+    flops = 4.0 * len(rsel) * w.n_tokens * w.head_dim
+    desc = (f"one (batch, head) slice of {w.name}: quantize+pack+unpack+dequant of K and V "
+            f"({w.n_tokens} tokens x {w.head_dim} channels), fp64 attention of {len(rsel)} query rows")
+    return dt, flops, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    rows = args.oracle_rows
+    times, flops = [], 0.0
+    desc = ""
+    for _ in range(args.warmup):
+        oracle_sample(w, args.bits, args.lq, rows)
+    for _ in range(args.steps):
+        dt, flops, desc = oracle_sample(w, args.bits, args.lq, rows)
+        times.append(dt)
+    tot = sum(times)
+    val = flops * len(times) / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, args):
+    return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} "
+                        f"blocks={w.n_blocks} Lq={args.lq} INT{args.bits}",
+            "global_batch": w.batch, "seq_len": w.n_tokens, "lq": args.lq, "bits": args.bits,
+            "parallelism": f"replica x{args.gpus}",
+            "l2": "inputs larger than L2 (bf16 K+V of the step exceed 126 MB)"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="infinity_8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--bits", type=int, default=4)
+    ap.add_argument("--also-bits", type=int, default=2, help="second bit width reported under 'also' (0: none)")
+    ap.add_argument("--lq", type=int, default=0, help="query block length (default: the workload's)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-rows", type=int, default=256)
+    ap.add_argument("--oracle-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    w = synth.WORKLOADS[args.workload]
+    if args.lq <= 0:
+        args.lq = w.lq[-1]
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    dist_ok = world > 1
+    if dist_ok:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+
+    def measure(bits):
+        pipe = Pipeline(w, bits, args.lq, dev)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(local)
+        sampler.start()
+        total_ms, qp, at = time_ours(pipe, args.steps, args.warmup, stream, dist_ok)
+        clocks = sampler.stop()
+        t = torch.tensor([total_ms], device=dev)
+        if dist_ok:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+        st = int(pipe.status.item())
+        return pipe, total_ms, qp, at, clocks, st
+
+    pipe, total_ms, qp, at, clocks, st = measure(args.bits)
+    flops = attention_flops(w, args.lq)
+    ms = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    at_avg = statistics.mean(at)
+    qp_avg = statistics.mean(qp)
+    att_tflops = flops / (at_avg * 1e-3) / 1e12
+    qbytes = quant_bytes(pipe.L, w)
+    qp_gbs = qbytes / (qp_avg * 1e-3) / 1e9
+    abytes = attention_bytes(pipe.L, w, args.lq, pipe.cos is not None)
+    tensor_peak = peaks["bf16_tflops_sustained"]
+    hbm_peak = peaks["hbm_gbs"]
+    roof_time = max(flops / (tensor_peak * 1e12), abytes / (hbm_peak * 1e9))
+    bound = "tensor" if flops / (tensor_peak * 1e12) >= abytes / (hbm_peak * 1e9) else "hbm"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 MMA / fp32 accumulate; int codes", "data": "synthetic",
+        "config": config_of(w, args),
+        "gpu_launches": pipe.launches_per_step * args.steps,
+        "device_status": st,
+        "components": {
+            "quant_pack": {"us": 1e3 * qp_avg, "GB/s": qp_gbs, "algorithmic_bytes": qbytes,
+                           "frac_hbm": qp_gbs / hbm_peak, "peak_GB/s": hbm_peak},
+            "attention": {"us": 1e3 * at_avg, "TFLOP/s": att_tflops, "flops": flops,
+                          "algorithmic_bytes": abytes, "bound": bound,
+                          "frac_of_binding_roofline": roof_time / (at_avg * 1e-3)},
+        },
+        "roofline": {"kernel": "attn_tc_kernel (fused packed-KV attention)", "bound": bound,
+                     "achieved": att_tflops if bound == "tensor" else abytes / (at_avg * 1e-3) / 1e9,
+                     "peak": tensor_peak if bound == "tensor" else hbm_peak,
+                     "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                     "frac": (att_tflops / tensor_peak) if bound == "tensor" else
+                     (abytes / (at_avg * 1e-3) / 1e9) / hbm_peak,
+                     "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
+                     "traffic": None},
+        "clocks": clocks,
+    }
+    if args.also_bits and args.also_bits != args.bits:
+        del pipe
+        torch.cuda.empty_cache()
+        p2, tot2, qp2, at2, clk2, st2 = measure(args.also_bits)
+        line["also"] = {
+            "bits": args.also_bits, "value": world * flops * args.steps / (tot2 * 1e-3) / 1e12,
+            "ms_per_step": tot2 / args.steps, "device_status": st2,
+            "quant_pack_GB/s": quant_bytes(p2.L, w) / (statistics.mean(qp2) * 1e-3) / 1e9,
+            "attention_TFLOP/s": flops / (statistics.mean(at2) * 1e-3) / 1e12,
+            "clocks": clk2}
+        line["also"]["quant_pack_frac_hbm"] = line["also"]["quant_pack_GB/s"] / hbm_peak
+        line["also"]["attention_frac_tensor"] = line["also"]["attention_TFLOP/s"] / tensor_peak
+        del p2
+        torch.cuda.empty_cache()
+        pipe = Pipeline(w, args.bits, args.lq, dev)
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(pipe, max(3, args.steps // 2), 2, stream)
+        line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # repeat the bounded sample (fresh seeds) for about ten seconds of CPU work
+        dt_tot, fl_tot, reps, desc = 0.0, 0.0, 0, ""
+        while dt_tot < args.oracle_seconds and reps < 64:
+            dt, sflops, desc = oracle_sample(w, args.bits, args.lq, args.oracle_rows, seed=reps)
+            dt_tot += dt
+            fl_tot += sflops
+            reps += 1
+        line["cpu_baseline"] = {"value": fl_tot / dt_tot / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} x [{desc}]", "seconds": dt_tot}
+    if dist_ok:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,218 @@
+/*
+ * varq.h -- C ABI of libvarq, the sm_100a (B200) implementation of the VAR-Q
+ * packed KV-cache hot path.
+ *
+ * What the library computes (sources are the VAR-Q pages):
+ *   - "VAR-Q: Tuning-free KV Cache Quantization for Visual Autoregressive
+ *     Image and Video Generation", project page  [PAGE]
+ *   - "VAR-Q: KV-Cache Quantization for Visual Autoregressive Generation",
+ *     repository README                          [README]
+ *
+ *   Quantization: one (scale, minimum) pair per (batch, head, channel,
+ *   generation block) cell; asymmetric min-max round-to-nearest-even codes of
+ *   b in [2, 8] bits ([PAGE] "Next-block prediction", "Channel x block
+ *   KV-cache quantization"):
+ *       s = fp32(fp32(max - min) / (2^b - 1))
+ *       q = clamp(rint(fp32(fp32(x - min) / s)), 0, 2^b - 1); q = 0 if s == 0
+ *   Packing: floor(32/b) codes of consecutive tokens of one channel per
+ *   uint32, least significant bits first, contiguous over the whole token
+ *   axis ([PAGE] "Quantization, bit packing, and retrieval": low-bit values
+ *   packed into INT32 storage).  3-bit packs 10 codes per word.
+ *   Metadata: one uint32 per cell, fp16(s) in bits 0-15 and fp16(min) in bits
+ *   16-31, never expanded over tokens ([README] "Memory-Efficient Runtime").
+ *   Dequantization: x_hat = bf16_rn(fmaf(q, s16, m16)) ([PAGE] "Quantization,
+ *   bit packing, and retrieval": unpacked and dequantized to BF16 before
+ *   attention).
+ *   Attention: O = softmax(scale * Q K_hat^T) V_hat over every cached token of
+ *   blocks [0, n_cached_blocks) ([PAGE] "Next-block prediction": every block
+ *   attends to the KV cache of all blocks before it), with the packed cache
+ *   read and dequantized inside the attention kernel ([README] "Fused-kernel
+ *   overhead reduction").
+ *
+ * Memory layouts (all row-major, element strides where stated):
+ *   packed cache  uint32 [B, H, W, D], W = ceil(T / floor(32/b)), contiguous
+ *   metadata      uint32 [B, H, NB, D], contiguous
+ *   K/V input     bf16, element (b, h, t, d) at x[b*sb + h*sh + t*st + d]
+ *   queries       bf16, element (b, h, i, d) at q[b*q_sb + h*q_sh + i*q_st + d]
+ *   output        bf16, same convention with o_sb, o_sh, o_st
+ *   RoPE tables   fp32 [T, D/2] contiguous (row t = cache token t)
+ *
+ * Ownership: the library allocates nothing and keeps no state between
+ * calls.  Every pointer is caller-owned; device pointers must stay valid
+ * until the work queued on `stream` has finished.  All calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream).  The library is thread-safe.
+ *
+ * Errors: host-detectable argument errors return a negative varq_status
+ * before anything is launched.  VARQ_ERR_CUDA reports a launch failure
+ * (cudaGetLastError after the launch).  Faults in the data (non-finite input,
+ * metadata out of fp16 range, a pipeline wait that timed out) are reported
+ * through the optional device status word `dev_status` (bits VARQ_DEV_*,
+ * set with atomicOr; the caller zeroes it and reads it after the stream
+ * work finishes); they never trap.
+ */
+#ifndef VARQ_H
+#define VARQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define VARQ_API __attribute__((visibility("default")))
+#else
+#define VARQ_API
+#endif
+
+#define VARQ_MAX_BLOCKS 256
+
+typedef enum varq_status {
+  VARQ_OK = 0,
+  VARQ_ERR_INVALID_ARG = -1,  /* a size, index or pointer is out of range   */
+  VARQ_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. D = 96)    */
+  VARQ_ERR_CUDA = -3,         /* the CUDA runtime reported an error         */
+  VARQ_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required */
+  VARQ_ERR_ALIGNMENT = -5     /* a pointer or stride breaks 16-byte rules   */
+} varq_status;
+
+/* Bits of the device status word. */
+#define VARQ_DEV_NONFINITE 1u      /* a quantized input value was NaN or Inf       */
+#define VARQ_DEV_META_OVERFLOW 2u  /* |min| or s exceeded the fp16 range (65504)   */
+#define VARQ_DEV_TIMEOUT 4u        /* an attention pipeline wait ran out; the call */
+                                   /* returned early and its output is undefined   */
+
+/* Attention path selection (the `path` argument of varq_packed_attention). */
+#define VARQ_PATH_AUTO 0           /* tensor-core path or split-KV path by Lq      */
+#define VARQ_PATH_TENSOR 1         /* tcgen05 path: 128 query rows per CTA         */
+#define VARQ_PATH_SPLIT 2          /* split-KV path (Lq <= VARQ_SPLIT_MAX_LQ)      */
+#define VARQ_SPLIT_MAX_LQ 16
+
+/*
+ * Plan of one packed cache tensor (K or V; both use the same plan).
+ * Filled by varq_cache_alloc; the other calls read it.
+ */
+typedef struct varq_cache_layout {
+  int32_t batch;            /* B >= 1                                         */
+  int32_t heads;            /* H >= 1                                         */
+  int32_t head_dim;         /* D in {64, 128}                                 */
+  int32_t bits;             /* b in [2, 8]                                    */
+  int32_t codes_per_word;   /* floor(32 / b)                                  */
+  int32_t n_blocks;         /* NB in [1, VARQ_MAX_BLOCKS]                     */
+  int64_t n_tokens;         /* T = block_start[NB]                            */
+  int64_t words_per_row;    /* W = ceil(T / codes_per_word)                   */
+  int64_t packed_bytes;     /* B * H * W * D * 4                              */
+  int64_t meta_bytes;       /* B * H * NB * D * 4                             */
+  int32_t block_start[VARQ_MAX_BLOCKS + 1]; /* token offsets; [0] = 0        */
+} varq_cache_layout;
+
+/*
+ * varq_cache_alloc -- exact preallocation plan ([README] "Memory-Efficient
+ * Runtime": packed K/V buffers preallocated when the generation length is
+ * known).  Pure host integer arithmetic; touches no GPU.
+ *
+ *   block_start  host array of n_blocks + 1 token offsets, block_start[0] = 0,
+ *                strictly increasing (the generation loop's block
+ *                boundaries: scales or frames).
+ *   out          filled on success.
+ * The caller allocates packed_bytes and meta_bytes of device memory per
+ * tensor (K and V each).  No zeroing is needed: quantization writes every bit
+ * a block owns.
+ * Returns VARQ_OK, VARQ_ERR_INVALID_ARG (bad sizes, offsets, NULL) or
+ * VARQ_ERR_UNSUPPORTED (head_dim not 64/128, n_blocks > VARQ_MAX_BLOCKS).
+ */
+VARQ_API int varq_cache_alloc(int batch, int heads, int head_dim, int bits,
+                     const int32_t* block_start, int n_blocks,
+                     varq_cache_layout* out);
+
+/*
+ * varq_quantize_pack -- quantize blocks [first_block, first_block + n_blocks)
+ * of K or V into the packed cache and its metadata ([PAGE] "Channel x block
+ * KV-cache quantization"; "Quantization, bit packing, and retrieval").
+ *
+ *   x            device bf16; row t of x is cache token
+ *                block_start[first_block] + t.  16-byte aligned; sb, sh, st
+ *                multiples of 8 elements; channels contiguous.
+ *   packed       device uint32 [B, H, W, D], 16-byte aligned.
+ *   meta         device uint32 [B, H, NB, D], 16-byte aligned.
+ *   dev_status   device uint32 or NULL (VARQ_DEV_NONFINITE,
+ *                VARQ_DEV_META_OVERFLOW).
+ * Every bit a block owns is rewritten: its codes, the padding slots past T if
+ * it is the last block, and bits 30-31 (or 28-31) of words whose first slot
+ * it owns.  Words shared with a neighbouring block are updated atomically,
+ * so blocks may be (re)quantized in any order and overwritten later.
+ * Calls that write the same block concurrently race.
+ */
+VARQ_API int varq_quantize_pack(const varq_cache_layout* layout, const void* x,
+                       int64_t sb, int64_t sh, int64_t st,
+                       int first_block, int n_blocks,
+                       uint32_t* packed, uint32_t* meta,
+                       uint32_t* dev_status, void* stream);
+
+/*
+ * varq_unpack_dequant -- standalone unpack + dequantize of blocks
+ * [first_block, first_block + n_blocks) to dense bf16 (the unfused path:
+ * [PAGE] "Quantization, bit packing, and retrieval"; [README] CUDA
+ * "unpack+dequant" operator).  Bit-exact x_hat = bf16_rn(fmaf(q, s16, m16)).
+ *
+ *   out          device bf16; row t is cache token block_start[first_block]
+ *                + t; 16-byte aligned, strides multiples of 8 elements.
+ */
+VARQ_API int varq_unpack_dequant(const varq_cache_layout* layout, const uint32_t* packed,
+                        const uint32_t* meta, int first_block, int n_blocks,
+                        void* out, int64_t sb, int64_t sh, int64_t st,
+                        void* stream);
+
+/*
+ * varq_packed_attention_workspace -- bytes of device workspace
+ * varq_packed_attention needs for this shape and path (0 if none).
+ */
+VARQ_API size_t varq_packed_attention_workspace(const varq_cache_layout* layout, int lq,
+                                       int n_cached_blocks, int path);
+
+/*
+ * varq_packed_attention -- attention of a query block over the packed cache,
+ * unpacking and dequantizing K and V inside the kernel ([README]
+ * "Fused-kernel overhead reduction"; [PAGE] "Next-block prediction").
+ *
+ *   q            device bf16 [B, H, lq, D] with strides q_sb, q_sh, q_st
+ *                (elements; multiples of 8; 16-byte aligned base).  Queries
+ *                arrive final (already rotated if the model uses RoPE).
+ *   k_packed, k_meta, v_packed, v_meta   the two caches (same layout).
+ *   n_cached_blocks  attend over tokens [0, block_start[n_cached_blocks]).
+ *   softmax_scale    <= 0 selects 1/sqrt(D).
+ *   rope_cos, rope_sin  NULL, or fp32 [T, D/2] tables: pre-RoPE key mode,
+ *                key pair (2i, 2i+1) of token t is rotated by (cos, sin)
+ *                [t, i] after dequantization ([PAGE] "The block axis",
+ *                Eq. 3 and Appendix F).  Both or neither.
+ *   out          device bf16 [B, H, lq, D], strides o_sb, o_sh, o_st.
+ *   lse          device fp32 [B, H, lq] (natural-log sum of exp of the scaled
+ *                scores) or NULL.
+ *   workspace    device memory of varq_packed_attention_workspace() bytes
+ *                (may be NULL when that is 0).
+ *   path         VARQ_PATH_AUTO, VARQ_PATH_TENSOR or VARQ_PATH_SPLIT.
+ *   dev_status   device uint32 or NULL (VARQ_DEV_TIMEOUT).
+ */
+VARQ_API int varq_packed_attention(const varq_cache_layout* layout,
+                          const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st, int lq,
+                          const uint32_t* k_packed, const uint32_t* k_meta,
+                          const uint32_t* v_packed, const uint32_t* v_meta,
+                          int n_cached_blocks, float softmax_scale,
+                          const float* rope_cos, const float* rope_sin,
+                          void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
+                          float* lse, void* workspace, size_t workspace_bytes,
+                          int path, uint32_t* dev_status, void* stream);
+
+/* Human-readable name of a varq_status value (static string). */
+VARQ_API const char* varq_status_string(int status);
+
+/* Library ABI version (incremented when a signature changes). */
+VARQ_API int varq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARQ_H */

@@ -1,0 +1,86 @@
+// Host-side declarations shared by the libvarq translation units: kernel
+// argument blocks (passed by value as kernel parameters) and launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/varq.h"
+
+namespace varq {
+
+// ---------------------------------------------------------- quantize+pack
+
+struct QuantArgs {
+  const __nv_bfloat16* x;  // row 0 = cache token block_start[first_block]
+  int64_t sb, sh, st;      // element strides of x
+  uint32_t* packed;        // [B, H, W, D]
+  uint32_t* meta;          // [B, H, NB, D]
+  uint32_t* dev_status;    // nullable
+  int64_t words_per_row;
+  int32_t batch, heads, head_dim, bits, n_blocks_total, n_tokens;
+  int32_t first_block, n_blocks;
+  int32_t staged;          // 1: slices staged in shared memory
+  int32_t block_start[VARQ_MAX_BLOCKS + 1];
+};
+
+struct QuantPlan {
+  int group;     // channels per work item (64, 32 or 16)
+  int cluster;   // CTAs per work item (1..8), one token slice each
+  size_t smem;   // dynamic shared memory per CTA
+  int staged;
+};
+
+QuantPlan plan_quant_pack(int head_dim, int bits, int max_block_len);
+cudaError_t launch_quant_pack(const QuantArgs& a, const QuantPlan& p, cudaStream_t stream);
+
+// --------------------------------------------------------- unpack+dequant
+
+struct UnpackArgs {
+  const uint32_t* packed;
+  const uint32_t* meta;
+  __nv_bfloat16* out;      // row 0 = cache token block_start[first_block]
+  int64_t sb, sh, st;
+  int64_t words_per_row;
+  int32_t batch, heads, head_dim, bits, n_blocks_total, n_tokens;
+  int32_t first_block, n_blocks;
+  int32_t block_start[VARQ_MAX_BLOCKS + 1];
+};
+
+cudaError_t launch_unpack_dequant(const UnpackArgs& a, cudaStream_t stream);
+
+// -------------------------------------------------------------- attention
+
+struct AttnArgs {
+  const __nv_bfloat16* q;
+  int64_t q_sb, q_sh, q_st;
+  const uint32_t* k_packed;
+  const uint32_t* k_meta;
+  const uint32_t* v_packed;
+  const uint32_t* v_meta;
+  const float* rope_cos;   // nullable: [T, D/2]
+  const float* rope_sin;
+  __nv_bfloat16* out;
+  int64_t o_sb, o_sh, o_st;
+  float* lse;              // nullable: [B, H, lq]
+  float* workspace;        // split-KV partials
+  uint32_t* dev_status;
+  int64_t words_per_row;
+  int32_t batch, heads, head_dim, bits, n_blocks_total;
+  int32_t lq;
+  int32_t n_cached_blocks;
+  int32_t t_att;           // attended tokens: block_start[n_cached_blocks]
+  float scale_log2;        // softmax scale * log2(e)
+  float scale;             // softmax scale
+  int32_t n_splits;        // split-KV only
+  int32_t block_start[VARQ_MAX_BLOCKS + 1];
+};
+
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attention_split(const AttnArgs& a, cudaStream_t stream);
+int split_kv_splits(const AttnArgs& a);
+size_t split_kv_workspace_bytes(int batch, int heads, int lq, int head_dim, int n_splits);
+
+}  // namespace varq

@@ -1,0 +1,234 @@
+// Host side of the C ABI declared in include/varq.h: argument validation,
+// layout planning and kernel dispatch.  No allocation, no global state.
+#include <cmath>
+#include <cstring>
+
+#include "kernels.h"
+
+namespace {
+
+using varq::AttnArgs;
+using varq::QuantArgs;
+using varq::UnpackArgs;
+
+constexpr int64_t kMaxTokens = int64_t(1) << 30;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return (s % 8) == 0; }
+
+int check_layout(const varq_cache_layout* L) {
+  if (L == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (L->batch < 1 || L->heads < 1) return VARQ_ERR_INVALID_ARG;
+  if (L->head_dim != 64 && L->head_dim != 128) return VARQ_ERR_UNSUPPORTED;
+  if (L->bits < 2 || L->bits > 8) return VARQ_ERR_INVALID_ARG;
+  if (L->codes_per_word != 32 / L->bits) return VARQ_ERR_INVALID_ARG;
+  if (L->n_blocks < 1 || L->n_blocks > VARQ_MAX_BLOCKS) return VARQ_ERR_INVALID_ARG;
+  if (L->block_start[0] != 0) return VARQ_ERR_INVALID_ARG;
+  for (int i = 0; i < L->n_blocks; ++i)
+    if (L->block_start[i + 1] <= L->block_start[i]) return VARQ_ERR_INVALID_ARG;
+  const int64_t T = L->block_start[L->n_blocks];
+  if (L->n_tokens != T || T > kMaxTokens) return VARQ_ERR_INVALID_ARG;
+  const int64_t W = (T + L->codes_per_word - 1) / L->codes_per_word;
+  if (L->words_per_row != W) return VARQ_ERR_INVALID_ARG;
+  return VARQ_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? VARQ_OK : VARQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int varq_abi_version(void) { return 1; }
+
+const char* varq_status_string(int status) {
+  switch (status) {
+    case VARQ_OK: return "VARQ_OK";
+    case VARQ_ERR_INVALID_ARG: return "VARQ_ERR_INVALID_ARG: a size, index or pointer is out of range";
+    case VARQ_ERR_UNSUPPORTED: return "VARQ_ERR_UNSUPPORTED: valid request the library does not implement";
+    case VARQ_ERR_CUDA: return "VARQ_ERR_CUDA: the CUDA runtime reported an error";
+    case VARQ_ERR_WORKSPACE: return "VARQ_ERR_WORKSPACE: workspace missing or too small";
+    case VARQ_ERR_ALIGNMENT: return "VARQ_ERR_ALIGNMENT: pointer or stride breaks the 16-byte rule";
+    default: return "unknown varq status";
+  }
+}
+
+int varq_cache_alloc(int batch, int heads, int head_dim, int bits, const int32_t* block_start, int n_blocks,
+                     varq_cache_layout* out) {
+  if (out == nullptr || block_start == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || bits < 2 || bits > 8 || n_blocks < 1) return VARQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return VARQ_ERR_UNSUPPORTED;
+  if (n_blocks > VARQ_MAX_BLOCKS) return VARQ_ERR_UNSUPPORTED;
+  if (block_start[0] != 0) return VARQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_blocks; ++i)
+    if (block_start[i + 1] <= block_start[i]) return VARQ_ERR_INVALID_ARG;
+  const int64_t T = block_start[n_blocks];
+  if (T > kMaxTokens) return VARQ_ERR_INVALID_ARG;
+  varq_cache_layout L;
+  std::memset(&L, 0, sizeof(L));
+  L.batch = batch;
+  L.heads = heads;
+  L.head_dim = head_dim;
+  L.bits = bits;
+  L.codes_per_word = 32 / bits;
+  L.n_blocks = n_blocks;
+  L.n_tokens = T;
+  L.words_per_row = (T + L.codes_per_word - 1) / L.codes_per_word;
+  L.packed_bytes = int64_t(batch) * heads * L.words_per_row * head_dim * 4;
+  L.meta_bytes = int64_t(batch) * heads * n_blocks * head_dim * 4;
+  for (int i = 0; i <= n_blocks; ++i) L.block_start[i] = block_start[i];
+  *out = L;
+  return VARQ_OK;
+}
+
+int varq_quantize_pack(const varq_cache_layout* L, const void* x, int64_t sb, int64_t sh, int64_t st,
+                       int first_block, int n_blocks, uint32_t* packed, uint32_t* meta, uint32_t* dev_status,
+                       void* stream) {
+  int rc = check_layout(L);
+  if (rc != VARQ_OK) return rc;
+  if (x == nullptr || packed == nullptr || meta == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (first_block < 0 || n_blocks < 1 || first_block + n_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(meta)) return VARQ_ERR_ALIGNMENT;
+  if (!stride_ok(sb) || !stride_ok(sh) || !stride_ok(st)) return VARQ_ERR_ALIGNMENT;
+  int max_len = 0;
+  for (int k = first_block; k < first_block + n_blocks; ++k) {
+    const int len = L->block_start[k + 1] - L->block_start[k];
+    if (len > max_len) max_len = len;
+  }
+  QuantArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.sb = sb;
+  a.sh = sh;
+  a.st = st;
+  a.packed = packed;
+  a.meta = meta;
+  a.dev_status = dev_status;
+  a.words_per_row = L->words_per_row;
+  a.batch = L->batch;
+  a.heads = L->heads;
+  a.head_dim = L->head_dim;
+  a.bits = L->bits;
+  a.n_blocks_total = L->n_blocks;
+  a.n_tokens = static_cast<int32_t>(L->n_tokens);
+  a.first_block = first_block;
+  a.n_blocks = n_blocks;
+  std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
+  const varq::QuantPlan plan = varq::plan_quant_pack(L->head_dim, L->bits, max_len);
+  return launch_status(varq::launch_quant_pack(a, plan, static_cast<cudaStream_t>(stream)));
+}
+
+int varq_unpack_dequant(const varq_cache_layout* L, const uint32_t* packed, const uint32_t* meta, int first_block,
+                        int n_blocks, void* out, int64_t sb, int64_t sh, int64_t st, void* stream) {
+  int rc = check_layout(L);
+  if (rc != VARQ_OK) return rc;
+  if (out == nullptr || packed == nullptr || meta == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (first_block < 0 || n_blocks < 1 || first_block + n_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(packed) || !aligned16(meta)) return VARQ_ERR_ALIGNMENT;
+  if (!stride_ok(sb) || !stride_ok(sh) || !stride_ok(st)) return VARQ_ERR_ALIGNMENT;
+  if (int64_t(L->batch) * L->heads > 65535) return VARQ_ERR_UNSUPPORTED;
+  UnpackArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.packed = packed;
+  a.meta = meta;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.sb = sb;
+  a.sh = sh;
+  a.st = st;
+  a.words_per_row = L->words_per_row;
+  a.batch = L->batch;
+  a.heads = L->heads;
+  a.head_dim = L->head_dim;
+  a.bits = L->bits;
+  a.n_blocks_total = L->n_blocks;
+  a.n_tokens = static_cast<int32_t>(L->n_tokens);
+  a.first_block = first_block;
+  a.n_blocks = n_blocks;
+  std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
+  return launch_status(varq::launch_unpack_dequant(a, static_cast<cudaStream_t>(stream)));
+}
+
+static int choose_path(int lq, int path) {
+  if (path == VARQ_PATH_AUTO) return lq <= VARQ_SPLIT_MAX_LQ ? VARQ_PATH_SPLIT : VARQ_PATH_TENSOR;
+  return path;
+}
+
+static void fill_attn(AttnArgs& a, const varq_cache_layout* L, int lq, int n_cached_blocks) {
+  std::memset(&a, 0, sizeof(a));
+  a.words_per_row = L->words_per_row;
+  a.batch = L->batch;
+  a.heads = L->heads;
+  a.head_dim = L->head_dim;
+  a.bits = L->bits;
+  a.n_blocks_total = L->n_blocks;
+  a.lq = lq;
+  a.n_cached_blocks = n_cached_blocks;
+  a.t_att = L->block_start[n_cached_blocks];
+  std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
+}
+
+size_t varq_packed_attention_workspace(const varq_cache_layout* L, int lq, int n_cached_blocks, int path) {
+  if (check_layout(L) != VARQ_OK || lq < 1 || n_cached_blocks < 1 || n_cached_blocks > L->n_blocks) return 0;
+  if (choose_path(lq, path) != VARQ_PATH_SPLIT || lq > VARQ_SPLIT_MAX_LQ) return 0;
+  AttnArgs a;
+  fill_attn(a, L, lq, n_cached_blocks);
+  return varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, varq::split_kv_splits(a));
+}
+
+int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st,
+                          int lq, const uint32_t* k_packed, const uint32_t* k_meta, const uint32_t* v_packed,
+                          const uint32_t* v_meta, int n_cached_blocks, float softmax_scale, const float* rope_cos,
+                          const float* rope_sin, void* out, int64_t o_sb, int64_t o_sh, int64_t o_st, float* lse,
+                          void* workspace, size_t workspace_bytes, int path, uint32_t* dev_status, void* stream) {
+  int rc = check_layout(L);
+  if (rc != VARQ_OK) return rc;
+  if (q == nullptr || out == nullptr || k_packed == nullptr || k_meta == nullptr || v_packed == nullptr ||
+      v_meta == nullptr)
+    return VARQ_ERR_INVALID_ARG;
+  if (lq < 1 || n_cached_blocks < 1 || n_cached_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return VARQ_ERR_INVALID_ARG;
+  if (path != VARQ_PATH_AUTO && path != VARQ_PATH_TENSOR && path != VARQ_PATH_SPLIT) return VARQ_ERR_INVALID_ARG;
+  if (!(std::isfinite(softmax_scale))) return VARQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(k_meta) || !aligned16(v_packed) ||
+      !aligned16(v_meta))
+    return VARQ_ERR_ALIGNMENT;
+  if (!stride_ok(q_sb) || !stride_ok(q_sh) || !stride_ok(q_st) || !stride_ok(o_sb) || !stride_ok(o_sh) ||
+      !stride_ok(o_st))
+    return VARQ_ERR_ALIGNMENT;
+  if (L->heads > 65535 || L->batch > 65535) return VARQ_ERR_UNSUPPORTED;
+  const int p = choose_path(lq, path);
+  if (p == VARQ_PATH_SPLIT && lq > VARQ_SPLIT_MAX_LQ) return VARQ_ERR_UNSUPPORTED;
+
+  AttnArgs a;
+  fill_attn(a, L, lq, n_cached_blocks);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.q_sb = q_sb;
+  a.q_sh = q_sh;
+  a.q_st = q_st;
+  a.k_packed = k_packed;
+  a.k_meta = k_meta;
+  a.v_packed = v_packed;
+  a.v_meta = v_meta;
+  a.rope_cos = rope_cos;
+  a.rope_sin = rope_sin;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.o_sb = o_sb;
+  a.o_sh = o_sh;
+  a.o_st = o_st;
+  a.lse = lse;
+  a.dev_status = dev_status;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(float(L->head_dim));
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p == VARQ_PATH_TENSOR) return launch_status(varq::launch_attention_tc(a, s));
+
+  a.n_splits = varq::split_kv_splits(a);
+  const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits);
+  if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
+  a.workspace = static_cast<float*>(workspace);
+  return launch_status(varq::launch_attention_split(a, s));
+}
+
+}  // extern "C"
