@@ -24,6 +24,7 @@
 //   Q  [D/64 panels][128 rows][64]   K-major A of S = Q K^T
 //   K  [NKV/64 panels][D rows][64]   row = channel, columns = tokens:
 //                                    MN-major B of S = Q K^T
+// Q and K are fp16 instead of bf16 in the pre-RoPE key mode (see QK_F16).
 //   V  [NKV/64 panels][D rows][64]   same storage, read as K-major B of
 //                                    O = P V (N = channel, K = token)
 //   P  [NKV/64 panels][128 rows][64] K-major A of O = P V
@@ -109,6 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   using C = Cfg<BITS, D>;
   constexpr int CPW = C::CPW;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
+  // Pre-RoPE keys are rotated after dequantization and must be rounded again
+  // for the MMA; fp16 (11-bit significand) keeps that rounding 8x below a
+  // bf16 ulp, so S = Q K^T runs in fp16 there (queries convert exactly).
+  constexpr bool QK_F16 = ROPE;
 
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -157,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int row = qtile * BM + r;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row < a.lq) v = __ldg(reinterpret_cast<const uint4*>(qg + int64_t(row) * a.q_st + c * 8));
+      if (QK_F16) v = bf16x8_to_f16x8(v);
       *reinterpret_cast<uint4*>(smem + C::OFF_Q + sw128_offset(r, c * 8, BM)) = v;
     }
     fence_async_smem();
@@ -204,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, C::NKV, false, true);
+      constexpr uint32_t idesc_qk =
+          QK_F16 ? idesc_f16_f32(BM, C::NKV, false, true) : idesc_bf16_f32(BM, C::NKV, false, true);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, false);
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t k_base = smem_u32(smem + C::OFF_K);
@@ -331,7 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < C::GC; ++c) {
             uint32_t pk[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) pk[i] = pack_bf16x2(x[c * 8 + 2 * i], x[c * 8 + 2 * i + 1]);
+            for (int i = 0; i < 4; ++i)
+              pk[i] = (QK_F16 && tensor == 0) ? pack_f16x2(x[c * 8 + 2 * i], x[c * 8 + 2 * i + 1])
+                                              : pack_bf16x2(x[c * 8 + 2 * i], x[c * 8 + 2 * i + 1]);
             const int tt = g * C::GT + c * 8;  // token within the tile
             const uint32_t off = (tt >> 6) * (D * 128) + ((((tt >> 3) & 7) ^ (d & 7)) << 4);
             *reinterpret_cast<uint4*>(dst + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);

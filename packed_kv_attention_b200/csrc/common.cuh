@@ -197,6 +197,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool a_mn_ma
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t(n) >> 3) << 17) | ((uint32_t(m) >> 4) << 24);
 }
 
+// Same with fp16 A/B (format code 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t(n) >> 3) << 17) | ((uint32_t(m) >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle.  Bits [0,14) start
 // address >> 4, [16,30) leading-dimension byte offset >> 4, [32,46) stride
 // byte offset >> 4, [46,48) version (1), [61,64) layout (2 = 128B swizzle).
@@ -237,6 +243,20 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 8 bf16 (one 16-byte chunk) -> 8 fp16; exact for |x| in [2^-14, 65504].
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = pack_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // fp16 bit patterns of one metadata word -> (scale, minimum) in fp32.

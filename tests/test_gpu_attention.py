@@ -54,6 +54,14 @@ def _gpu_attention(L, k, v, q, n_cached, cos=None, sin=None, path=V.PATH_AUTO, w
 
 
 def _oracle_attention(k, v, q, bs, bits, n_cached, b, h, rows, cos=None, sin=None, scale=None):
+    """Oracle output and LSE of the selected rows, plus the LSE tolerance.
+
+    LSE is 1-Lipschitz in the max-norm of the scores, so its error is bounded
+    by the largest score error.  With pre-RoPE keys the rotated key is rounded
+    to fp16 for the MMA (half an ulp: 2^-11 relative), giving a score error of
+    at most scale * 2^-11 * sum_d |q_d| |k_td|; other roundings (fp32
+    accumulation, the exp2 approximation) are covered by 1e-3.
+    """
     t_att = bs[n_cached]
     kb = bf16_bits(k[b:b + 1, h:h + 1])
     vb = bf16_bits(v[b:b + 1, h:h + 1])
@@ -62,9 +70,17 @@ def _oracle_attention(k, v, q, bs, bits, n_cached, b, h, rows, cos=None, sin=Non
     khat = O.dequantize(kc, km, bs)[0, 0, :t_att]
     vhat = O.dequantize(vc, vm, bs)[0, 0, :t_att]
     qb = bf16_bits(q[b, h])
-    return O.attention(qb, khat, vhat, scale=scale,
-                       rope_cos=None if cos is None else cos.numpy()[:t_att],
-                       rope_sin=None if sin is None else sin.numpy()[:t_att], rows=rows)
+    cs = None if cos is None else cos.numpy()[:t_att]
+    sn = None if sin is None else sin.numpy()[:t_att]
+    o, lse = O.attention(qb, khat, vhat, scale=scale, rope_cos=cs, rope_sin=sn, rows=rows)
+    tol = np.full(len(lse), 1e-3)
+    if cs is not None:
+        d = qb.shape[-1]
+        sc = (1.0 / math.sqrt(d)) if scale is None else scale
+        kr = np.abs(O.rope_rotate(O.bf16_to_f32(khat), cs, sn))
+        qa = np.abs(O.bf16_to_f32(qb).astype(np.float64)[rows])
+        tol += sc * 2.0 ** -11 * (qa @ kr.T).max(axis=1)
+    return o, (lse, tol)
 
 
 def _check(out, lse, ref, ref_lse, b, h, rows):
@@ -73,7 +89,8 @@ def _check(out, lse, ref, ref_lse, b, h, rows):
     assert mx <= MAX_REL and mean <= MEAN_REL, (mx, mean)
     if lse is not None:
         l = lse[b, h].cpu().numpy()[rows]
-        assert np.max(np.abs(l - ref_lse)) <= 1e-2, np.max(np.abs(l - ref_lse))
+        want, tol = ref_lse
+        assert np.all(np.abs(l - want) <= tol), float(np.max(np.abs(l - want) - tol))
 
 
 CASES = [
