@@ -205,6 +205,38 @@ VARQ_API int varq_packed_attention(const varq_cache_layout* layout,
                           float* lse, void* workspace, size_t workspace_bytes,
                           int path, uint32_t* dev_status, void* stream);
 
+/*
+ * varq_packed_attention_noalloc -- the split-KV attention of
+ * varq_packed_attention (VARQ_PATH_SPLIT, lq <= VARQ_SPLIT_MAX_LQ) for
+ * callers that cannot allocate device memory: a process whose allocator has
+ * already reserved the device memory for its own pool, code that is handed
+ * tensors but no allocator, or a loop that cannot afford cudaMalloc's implicit
+ * device synchronisation.  The pages have no counterpart of this entry point.
+ *
+ * Same arguments as varq_packed_attention without workspace, workspace_bytes
+ * and path.  The split partials live in a fixed array of
+ * VARQ_NOALLOC_SCRATCH_BYTES that the library keeps in the memory of every
+ * GPU that loads it, until the process exits; the caller still passes all
+ * inputs and outputs.  Nothing is allocated or freed.
+ *   - The first call on a device looks up that array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture begins.  Call with the device that owns `stream` current.
+ *   - Every call shares the one array: calls whose GPU work overlaps (other
+ *     streams, other threads) race.  Serialise them.
+ *   - A shape whose partials need more than VARQ_NOALLOC_SCRATCH_BYTES
+ *     (varq_packed_attention_workspace(..., VARQ_PATH_SPLIT) tells how much)
+ *     returns VARQ_ERR_WORKSPACE before anything is launched.
+ */
+#define VARQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+VARQ_API int varq_packed_attention_noalloc(const varq_cache_layout* layout,
+                                           const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st, int lq,
+                                           const uint32_t* k_packed, const uint32_t* k_meta,
+                                           const uint32_t* v_packed, const uint32_t* v_meta,
+                                           int n_cached_blocks, float softmax_scale,
+                                           const float* rope_cos, const float* rope_sin,
+                                           void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
+                                           float* lse, uint32_t* dev_status, void* stream);
+
 /* Human-readable name of a varq_status value (static string). */
 VARQ_API const char* varq_status_string(int status);
 

@@ -19,6 +19,7 @@ __all__ = [
     "varq_status_string", "varq_abi_version", "alloc_cache", "MAX_BLOCKS",
     "PATH_AUTO", "PATH_TENSOR", "PATH_SPLIT", "SPLIT_MAX_LQ",
     "DEV_NONFINITE", "DEV_META_OVERFLOW", "DEV_TIMEOUT",
+    "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvarq.so")
@@ -209,3 +210,36 @@ def varq_packed_attention(layout: CacheLayout, q: torch.Tensor, k_packed: torch.
         _ptr(rope_cos), _ptr(rope_sin), _ptr(out), out.stride(0), out.stride(1), out.stride(2),
         _ptr(lse), _ptr(workspace), ws_bytes, path, _ptr(dev_status), _stream(stream))
     _check(rc, "varq_packed_attention")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def varq_packed_attention_noalloc(layout: CacheLayout, q: torch.Tensor, k_packed: torch.Tensor,
+                                  k_meta: torch.Tensor, v_packed: torch.Tensor, v_meta: torch.Tensor,
+                                  out: torch.Tensor, n_cached_blocks: Optional[int] = None,
+                                  softmax_scale: float = 0.0, rope_cos: Optional[torch.Tensor] = None,
+                                  rope_sin: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                                  dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Split-KV attention (lq <= SPLIT_MAX_LQ) that allocates nothing: for
+    callers that cannot call cudaMalloc (their allocator already owns the
+    device memory, or the allocation's implicit synchronisation is not
+    acceptable).  The partials use the library's fixed per-device scratch
+    array of NOALLOC_SCRATCH_BYTES; calls must not overlap on the GPU."""
+    L = lib()
+    fn = L.varq_packed_attention_noalloc
+    fn.argtypes = [ctypes.POINTER(CacheLayout), _c_p, _c_i64, _c_i64, _c_i64, _c_int,
+                   _c_p, _c_p, _c_p, _c_p, _c_int, _c_f, _c_p, _c_p,
+                   _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_p]
+    fn.restype = _c_int
+    if n_cached_blocks is None:
+        n_cached_blocks = layout.n_blocks
+    _need(q, "q", torch.bfloat16)
+    _need(out, "out", torch.bfloat16)
+    if q.dim() != 4 or q.stride(3) != 1 or out.dim() != 4 or out.stride(3) != 1:
+        raise ValueError("q and out must be [B, H, lq, D] with contiguous channels")
+    rc = fn(ctypes.byref(layout), _ptr(q), q.stride(0), q.stride(1), q.stride(2), q.shape[2],
+            _ptr(k_packed), _ptr(k_meta), _ptr(v_packed), _ptr(v_meta), n_cached_blocks, float(softmax_scale),
+            _ptr(rope_cos), _ptr(rope_sin), _ptr(out), out.stride(0), out.stride(1), out.stride(2),
+            _ptr(lse), _ptr(dev_status), _stream(stream))
+    _check(rc, "varq_packed_attention_noalloc")
