@@ -7,29 +7,35 @@
 // values unpacked and dequantized to BF16 before attention; "Next-block
 // prediction": the query block attends to the KV cache of all blocks).
 //
-// One CTA = 128 query rows of one (batch, head).  Warp roles:
-//   warps 0-3  softmax: one query row per thread (TMEM lane), online softmax
-//              in the log2 domain, P written to shared memory as bf16,
-//              O rescaled in TMEM, epilogue.
-//   warps 4-7  dequant: one channel per thread; packed words + per-block
-//              (scale, min) -> bf16, written straight into the 128-byte
-//              swizzled operand layout the MMA reads (optionally rotating
-//              key pairs for the pre-RoPE key mode).
-//   warp 8     producer: 1-D bulk copies (TMA engine) of the packed K/V words
-//              and of the metadata rows a tile touches, mbarrier completion.
-//   warp 9     MMA issuer: S = Q K^T into a double-buffered TMEM tile,
-//              O += P V into a TMEM accumulator, tcgen05.commit to mbarriers.
+// One CTA = NQ query tiles of 128 rows (NQ = 2 for large query blocks) of one
+// (batch, head); every dequantized K/V tile feeds all NQ tiles.  Warp roles:
+//   warps 0-7   softmax: warpgroup i owns query tile i, one row per thread
+//               (= TMEM lane); online softmax in the log2 domain; P is written
+//               back into TMEM over the consumed S columns (16-bit pairs) and
+//               O is rescaled in TMEM only when the row max grows by > 2^8.
+//   warps 8-15  dequant: (channel, part of the tile) per thread; packed words
+//               + per-block (scale, min) -> exact bf16 values written straight
+//               into the 128-byte swizzled operand layout the MMA reads
+//               (optionally rotating key pairs for the pre-RoPE key mode).
+//   warp 16     producer: 1-D bulk copies (TMA engine) of the packed K/V
+//               word rows of a tile (and of metadata rows when shared
+//               memory allows), mbarrier transaction counts.
+//   warp 17     MMA issuer: S_i = Q_i K^T into TMEM, O_i += P_i V with P read
+//               from TMEM, tcgen05.commit to mbarriers.  Issue order per KV
+//               tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax
+//               warpgroup works while the tensor core runs the other tile.
+//               QK_i(j+1) overwrites the TMEM columns PV_i(j) reads P from;
+//               the MMAs of one issuing thread execute in order.
 //
-// Shared-memory operand layouts (bf16, 128-byte swizzle, 64 elements/row):
-//   Q  [D/64 panels][128 rows][64]   K-major A of S = Q K^T
-//   K  [NKV/64 panels][D rows][64]   row = channel, columns = tokens:
+// Shared-memory operand layouts (16-bit, 128-byte swizzle, 64 elements/row):
+//   Q_i [D/64 panels][128 rows][64]  K-major A of S_i = Q_i K^T
+//   K   [NKV/64 panels][D rows][64]  row = channel, columns = tokens:
 //                                    MN-major B of S = Q K^T
-// Q and K are fp16 instead of bf16 in the pre-RoPE key mode (see QK_F16).
-//   V  [NKV/64 panels][D rows][64]   same storage, read as K-major B of
+//   V   [NKV/64 panels][D rows][64]  same storage, read as K-major B of
 //                                    O = P V (N = channel, K = token)
-//   P  [NKV/64 panels][128 rows][64] K-major A of O = P V
 // One packed word holds consecutive tokens of one channel, so unpacking it
 // yields a contiguous run along a row of the K and V tiles in both GEMMs.
+// Q and K are fp16 instead of bf16 in the pre-RoPE key mode (QK_F16).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -37,62 +43,80 @@ namespace varq {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kSoftmaxWarp0 = 0;
-constexpr int kDequantWarp0 = 4;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 576;
+constexpr int kDequantWarp0 = 8;
+constexpr int kDequantThreads = 256;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int BM = 128;
-constexpr int kMetaRows = 8;              // metadata rows staged per tile and tensor
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 192, kColO = 384;
-constexpr float kRescaleThreshold = 8.0f; // log2 units: rescale O only when the max grows by > 2^8
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kSmemUsable = 227 * 1024 - 1024;  // minus 1 KB to align the base to 1024
+constexpr uint32_t kBarBytes = 2048;
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
 
-template <int BITS, int D>
+template <int BITS, int D, int NQ>
 struct Cfg {
   static constexpr int CPW = 32 / BITS;
-  static constexpr int GT = clcm(CPW, 8);            // tokens per dequant group (whole words, whole 16 B chunks)
-  static constexpr int GW = GT / CPW;                // words per group
-  static constexpr int GC = GT / 8;                  // 16-byte chunks per group
+  static constexpr int GT = clcm(CPW, 8);             // tokens per dequant group (whole words, whole chunks)
+  static constexpr int GW = GT / CPW;                 // words per group
+  static constexpr int GC = GT / 8;                   // 16-byte chunks per group
   static constexpr int UNIT = clcm(CPW, 16);
-  static constexpr int NKV = ((128 + UNIT - 1) / UNIT) * UNIT;  // tokens per KV tile (128..160)
-  static constexpr int NW = NKV / CPW;               // packed words per tile
-  static constexpr int NG = NKV / GT;                // groups per tile
+  static constexpr int NKV = (128 / UNIT) * UNIT;     // tokens per KV tile: 128, 96 (5-bit) or 80 (3/6-bit)
+  static constexpr int NW = NKV / CPW;                // packed words per tile
+  static constexpr int NG = NKV / GT;                 // dequant groups per tile
   static constexpr int PANELS = (NKV + 63) / 64;
-  static constexpr int TPC = 128 / D;                // dequant threads per channel
-  static constexpr uint32_t Q_BYTES = (D / 64) * BM * 128;
-  static constexpr uint32_t KV_BYTES = PANELS * D * 128;   // one bf16 K or V tile
-  static constexpr uint32_t P_BYTES = PANELS * BM * 128;
-  static constexpr uint32_t WORDS_BYTES = NW * D * 4;      // packed words of one tensor per tile
-  static constexpr uint32_t META_BYTES = kMetaRows * D * 4;
-  static constexpr uint32_t STAGE_BYTES = 2 * WORDS_BYTES + 2 * META_BYTES;
-  static constexpr uint32_t total(int pst, int kst) {
-    return Q_BYTES + kst * KV_BYTES + KV_BYTES + P_BYTES + pst * STAGE_BYTES + 2048 /*barriers, tables*/;
+  static constexpr int TPC = kDequantThreads / D;     // dequant threads per channel
+  // codes of a word are taken CPC at a time from a shifted copy, so their
+  // bit offsets inside it stay below 2^14
+  static constexpr int CPC = BITS == 2 ? 4 : (BITS == 3 ? 3 : (BITS == 8 ? 1 : 2));
+  static constexpr uint32_t Q_TILE_BYTES = (D / 64) * BM * 128;
+  static constexpr uint32_t Q_BYTES = NQ * Q_TILE_BYTES;
+  static constexpr uint32_t KV_BYTES = PANELS * D * 128;
+  static constexpr uint32_t WORDS_BYTES = NW * D * 4;
+  static constexpr uint32_t need(int pst, int kst, int vst, int rows) {
+    return Q_BYTES + (kst + vst) * KV_BYTES + pst * (2 * WORDS_BYTES + 2 * rows * D * 4) + kBarBytes;
   }
-  static constexpr int PST = (total(2, 2) <= kSmemLimit || total(2, 1) <= kSmemLimit) ? 2 : 1;
-  static constexpr int KST = total(PST, 2) <= kSmemLimit ? 2 : 1;
-  // byte offsets (1024-aligned operand tiles first)
+  // buffer counts: prefer 2 packed stages, then double-buffered K and V,
+  // then as many staged metadata rows (<= 8) as fit
+  static constexpr int pick() {
+    const int opts[5][3] = {{2, 2, 2}, {2, 2, 1}, {1, 2, 2}, {2, 1, 1}, {1, 1, 1}};
+    for (int o = 0; o < 5; ++o)
+      for (int r = 8; r >= 0; --r)
+        if (need(opts[o][0], opts[o][1], opts[o][2], r) <= kSmemUsable) return o * 16 + r;
+    return -1;
+  }
+  static constexpr int PICK = pick();
+  static_assert(PICK >= 0, "shared memory budget");
+  static constexpr int OPT = PICK / 16;
+  static constexpr int PST = (OPT == 2 || OPT == 4) ? 1 : 2;
+  static constexpr int KST = (OPT == 3 || OPT == 4) ? 1 : 2;
+  static constexpr int VST = (OPT == 0 || OPT == 2) ? 2 : 1;
+  static constexpr int META_ROWS = PICK % 16;
+  static constexpr uint32_t META_BYTES = META_ROWS * D * 4;
+  static constexpr uint32_t STAGE_BYTES = 2 * WORDS_BYTES + 2 * META_BYTES;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + KV_BYTES;
-  static constexpr uint32_t OFF_STAGE = OFF_P + P_BYTES;
+  static constexpr uint32_t OFF_STAGE = OFF_V + VST * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_STAGE + PST * STAGE_BYTES;
-  static constexpr uint32_t SMEM = OFF_BAR + 2048 + 1024 /*alignment slack*/;
-  static_assert(NKV % 16 == 0 && NKV <= 192, "tile shape");
-  static_assert(SMEM <= kSmemLimit + 1024, "shared memory budget");
+  static constexpr uint32_t SMEM = OFF_BAR + kBarBytes + 1024;
+  static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
+  static_assert(NKV % 16 == 0 && NKV <= 128, "tile shape");
 };
 
+__host__ __device__ constexpr uint32_t col_s(int i) { return uint32_t(i) * 128u; }
+template <int NQ>
+__host__ __device__ constexpr uint32_t col_o(int i) { return uint32_t(NQ) * 128u + uint32_t(i) * 128u; }
+
 struct Barriers {
-  uint64_t full[2], empty[2];   // packed stage filled by TMA / released by dequant
-  uint64_t kready[2], kfree[2]; // bf16 K tile written / consumed by the S MMA
-  uint64_t vready, vfree;       // bf16 V tile written / consumed by the PV MMA
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_ready, o_done;
+  uint64_t full[2], empty[2];     // packed stage filled by TMA / released by dequant
+  uint64_t kready[2], kfree[2];   // 16-bit K tile written / consumed by all S MMAs
+  uint64_t vready[2], vfree[2];   // 16-bit V tile written / consumed by all PV MMAs
+  uint64_t s_full[2];             // S_i of the current tile in TMEM
+  uint64_t p_ready[2];            // P_i in TMEM and O_i rescaled
+  uint64_t o_done[2];             // PV_i finished
   uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
@@ -105,9 +129,9 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
 
 }  // namespace
 
-template <int BITS, int D, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnArgs a) {
-  using C = Cfg<BITS, D>;
+  using C = Cfg<BITS, D, NQ>;
   constexpr int CPW = C::CPW;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   // Pre-RoPE keys are rotated after dequantization and must be rounded again
@@ -123,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int qtile = blockIdx.x;
+  const int qblk = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int t_att = a.t_att;
@@ -134,36 +158,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->full[i], 1);
-      mbar_init(&bars->empty[i], 128);
-      mbar_init(&bars->kready[i], 128);
+      mbar_init(&bars->empty[i], kDequantThreads);
+      mbar_init(&bars->kready[i], kDequantThreads);
       mbar_init(&bars->kfree[i], 1);
+      mbar_init(&bars->vready[i], kDequantThreads);
+      mbar_init(&bars->vfree[i], 1);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 128);
+      mbar_init(&bars->p_ready[i], 128);
+      mbar_init(&bars->o_done[i], 1);
     }
-    mbar_init(&bars->vready, 128);
-    mbar_init(&bars->vfree, 1);
-    mbar_init(&bars->p_ready, 128);
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->teardown, 1);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
   for (int i = tid; i <= a.n_cached_blocks; i += kThreads) sm_bs[i] = a.block_start[i];
   if (warp == kMmaWarp) {
-    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  // Q tile -> K-major swizzled smem (rows past lq are zero)
+  // query tiles -> K-major swizzled smem (rows past lq are zero)
   {
     const __nv_bfloat16* qg = a.q + int64_t(b) * a.q_sb + int64_t(h) * a.q_sh;
     constexpr int CH = D / 8;
-    for (int i = tid; i < BM * CH; i += kThreads) {
-      const int r = i / CH, c = i % CH;
-      const int row = qtile * BM + r;
+    for (int idx = tid; idx < NQ * BM * CH; idx += kThreads) {
+      const int r = idx / CH, c = idx % CH;
+      const int row = qblk * (NQ * BM) + r;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row < a.lq) v = __ldg(reinterpret_cast<const uint4*>(qg + int64_t(row) * a.q_st + c * 8));
       if (QK_F16) v = bf16x8_to_f16x8(v);
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + sw128_offset(r, c * 8, BM)) = v;
+      *reinterpret_cast<uint4*>(smem + C::OFF_Q + (r / BM) * C::Q_TILE_BYTES + sw128_offset(r % BM, c * 8, BM)) = v;
     }
     fence_async_smem();
   }
@@ -187,20 +210,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, abort_flag)) break;
         const int w0 = j * C::NW;
         const int nw = min(C::NW, words_att - w0);
-        const int tok0 = w0 * CPW;
-        const int tok1 = min(tok0 + C::NKV, t_att);
-        while (tok0 >= sm_bs[blk + 1]) ++blk;
-        int blk_hi = blk;
-        while (tok1 - 1 >= sm_bs[blk_hi + 1]) ++blk_hi;
-        const int nrows = min(blk_hi - blk + 1, kMetaRows);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
         const uint32_t wbytes = uint32_t(nw) * D * 4;
-        const uint32_t mbytes = uint32_t(nrows) * D * 4;
+        uint32_t mbytes = 0;
+        int blk_lo = blk;
+        if (C::META_ROWS > 0) {
+          const int tok0 = w0 * CPW;
+          const int tok1 = min(tok0 + C::NKV, t_att);
+          while (tok0 >= sm_bs[blk + 1]) ++blk;
+          blk_lo = blk;
+          int blk_hi = blk;
+          while (tok1 - 1 >= sm_bs[blk_hi + 1]) ++blk_hi;
+          mbytes = uint32_t(min(blk_hi - blk_lo + 1, C::META_ROWS)) * D * 4;
+        }
         mbar_arrive_expect_tx(&bars->full[st], 2 * wbytes + 2 * mbytes);
         bulk_g2s(sb, kw + int64_t(w0) * D, wbytes, &bars->full[st]);
         bulk_g2s(sb + C::WORDS_BYTES, vw + int64_t(w0) * D, wbytes, &bars->full[st]);
-        bulk_g2s(sb + 2 * C::WORDS_BYTES, km + int64_t(blk) * D, mbytes, &bars->full[st]);
-        bulk_g2s(sb + 2 * C::WORDS_BYTES + C::META_BYTES, vm + int64_t(blk) * D, mbytes, &bars->full[st]);
+        if (C::META_ROWS > 0) {
+          bulk_g2s(sb + 2 * C::WORDS_BYTES, km + int64_t(blk_lo) * D, mbytes, &bars->full[st]);
+          bulk_g2s(sb + 2 * C::WORDS_BYTES + C::META_BYTES, vm + int64_t(blk_lo) * D, mbytes, &bars->full[st]);
+        }
         issued = j + 1;
       }
       // never leave copies in flight: wait for every stage that was filled
@@ -216,90 +245,121 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t k_base = smem_u32(smem + C::OFF_K);
       const uint32_t v_base = smem_u32(smem + C::OFF_V);
-      const uint32_t p_base = smem_u32(smem + C::OFF_P);
-      bool ok = true;
-      for (int j = 0; j <= ntiles && ok; ++j) {
-        if (j < ntiles) {
-          const int ks = j % C::KST;
-          const int sbuf = j & 1;
-          ok = mbar_wait(&bars->kready[ks], (j / C::KST) & 1, abort_flag);
-          if (ok && j >= 2) ok = mbar_wait(&bars->s_free[sbuf], ((j >> 1) - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + (sbuf ? kColS1 : kColS0);
+      auto issue_qk = [&](int i, int j) {
+        const uint32_t kb = k_base + (j % C::KST) * C::KV_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(q_base + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(k_base + ks * C::KV_BYTES + kk * 2048, D * 128, 1024);
-            mma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->s_full[sbuf]);
-          mma_commit(&bars->kfree[ks]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad =
+              smem_desc_sw128(q_base + i * C::Q_TILE_BYTES + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(kb + kk * 2048, D * 128, 1024);
+          mma_ss(tmem + col_s(i), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int i = j - 1;
-          ok = mbar_wait(&bars->p_ready, i & 1, abort_flag);
-          if (ok) ok = mbar_wait(&bars->vready, i & 1, abort_flag);
+      };
+      auto issue_pv = [&](int i, int j) {
+        const uint32_t vb = v_base + (j % C::VST) * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::NKV / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(vb + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024);
+          mma_ts(tmem + col_o<NQ>(i), tmem + col_s(i) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bars->kready[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < NQ; ++i) {
+          issue_qk(i, 0);
+          mma_commit(&bars->s_full[i]);
+        }
+        mma_commit(&bars->kfree[0]);
+      }
+      for (int j = 0; j < ntiles && ok; ++j) {
+        ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag);
+        for (int i = 0; i < NQ && ok; ++i) {
+          ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::NKV / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(p_base + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(v_base + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024);
-            mma_ss(tmem + kColO, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          issue_pv(i, j);
+          mma_commit(&bars->o_done[i]);
+          if (i == NQ - 1) mma_commit(&bars->vfree[j % C::VST]);
+          if (j + 1 < ntiles) {
+            if (i == 0) {
+              ok = mbar_wait(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_qk(i, j + 1);
+            mma_commit(&bars->s_full[i]);
+            if (i == NQ - 1) mma_commit(&bars->kfree[(j + 1) % C::KST]);
           }
-          mma_commit(&bars->o_done);
-          mma_commit(&bars->vfree);
         }
       }
       // every MMA issued so far has finished before TMEM is released
       mma_commit(&bars->teardown);
       mbar_wait(&bars->teardown, 0, abort_flag);
     }
-  } else if (warp >= kDequantWarp0 && warp < kDequantWarp0 + 4) {
+  } else if (warp >= kDequantWarp0) {
     // ------------------------------------------------------------- dequant
     const int dt = tid - kDequantWarp0 * 32;
     const int d = dt % D;
     const int part = dt / D;
-    int blk = 0;  // block of the current token (monotone over tiles)
+    int blk = 0;  // block of the current tile's first token (monotone)
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % C::PST;
-      const int ks = j % C::KST;
       if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
       const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
       const int tok0 = j * C::NKV;
-      int blk_lo = blk;
-      while (tok0 >= sm_bs[blk_lo + 1]) ++blk_lo;
-      for (int tensor = 0; tensor < 2; ++tensor) {
-        if (tensor == 0) {
-          if (j >= C::KST && !wait_all(&bars->kfree[ks], ((j / C::KST) - 1) & 1, abort_flag)) break;
-        } else {
-          if (j >= 1 && !wait_all(&bars->vfree, (j - 1) & 1, abort_flag)) break;
+      while (tok0 >= sm_bs[blk + 1]) ++blk;
+      const int blk_lo = blk;
+      bool ok = true;
+      for (int tensor = 0; tensor < 2 && ok; ++tensor) {
+        const int nbuf = tensor == 0 ? C::KST : C::VST;
+        const int buf = j % nbuf;
+        uint64_t* freeb = tensor == 0 ? &bars->kfree[buf] : &bars->vfree[buf];
+        if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
         }
         const uint32_t* words = reinterpret_cast<const uint32_t*>(sb + tensor * C::WORDS_BYTES);
-        const uint32_t* mrows = reinterpret_cast<const uint32_t*>(sb + 2 * C::WORDS_BYTES + tensor * C::META_BYTES);
-        const uint32_t* mglob = (tensor == 0 ? a.k_meta : a.v_meta) +
-                                (int64_t(b) * a.heads + h) * a.n_blocks_total * D + d;
-        uint8_t* dst = smem + (tensor == 0 ? C::OFF_K + ks * C::KV_BYTES : C::OFF_V) + d * 128;
-        int cb = blk_lo;              // current block
-        int nb = sm_bs[cb + 1];       // its end
+        const uint32_t* mrows =
+            reinterpret_cast<const uint32_t*>(sb + 2 * C::WORDS_BYTES + tensor * C::META_BYTES);
+        const uint32_t* mglob =
+            (tensor == 0 ? a.k_meta : a.v_meta) + (int64_t(b) * a.heads + h) * a.n_blocks_total * D + d;
+        uint8_t* dst = smem + (tensor == 0 ? C::OFF_K : C::OFF_V) + buf * C::KV_BYTES + d * 128;
+        int cb = blk_lo;         // current block
+        int nb = sm_bs[cb + 1];  // its end
         auto meta_of = [&](int k) -> float2 {
-          const uint32_t w = (k - blk_lo < kMetaRows) ? mrows[(k - blk_lo) * D + d] : __ldg(mglob + int64_t(k) * D);
+          const uint32_t w =
+              (k - blk_lo < C::META_ROWS) ? mrows[(k - blk_lo) * D + d] : __ldg(mglob + int64_t(k) * D);
           return meta_unpack(w);
         };
         float2 sm = meta_of(cb);
+        // exact code -> value without a shift per code: the code at bit r of
+        // a shifted word becomes 2^23 + q 2^r (OR into the mantissa of 2^23),
+        // then fma(., s 2^-r, -2^(23-r) s) = q s exactly and + m rounds once,
+        // which is fmaf(q, s, m).
+        float cs[C::CPC], cc[C::CPC];
+        auto set_consts = [&](float s) {
+#pragma unroll
+          for (int rr = 0; rr < C::CPC; ++rr) {
+            cs[rr] = s * __uint_as_float(uint32_t(127 - rr * BITS) << 23);
+            cc[rr] = -s * __uint_as_float(uint32_t(127 + 23 - rr * BITS) << 23);
+          }
+        };
+        set_consts(sm.x);
         for (int g = part; g < C::NG; g += C::TPC) {
           const int tg = tok0 + g * C::GT;
           uint32_t wv[C::GW];
 #pragma unroll
           for (int i = 0; i < C::GW; ++i) wv[i] = words[(g * C::GW + i) * D + d];
           float x[C::GT];
-          const bool uniform = (tg + C::GT <= nb) && (tg + C::GT <= t_att);
-          if (uniform) {
+          if (tg + C::GT <= nb && tg + C::GT <= t_att) {
 #pragma unroll
             for (int jt = 0; jt < C::GT; ++jt) {
-              const uint32_t q = (wv[jt / CPW] >> ((jt % CPW) * BITS)) & MASK;
-              x[jt] = __fmaf_rn(small_uint_to_float(q), sm.x, sm.y);
+              const int jj = jt % CPW;
+              const int chunk = jj / C::CPC, rr = jj % C::CPC;
+              const uint32_t ws = wv[jt / CPW] >> (chunk * C::CPC * BITS);
+              const float f = __uint_as_float((ws & (MASK << (rr * BITS))) | 0x4B000000u);
+              x[jt] = __fadd_rn(__fmaf_rn(f, cs[rr], cc[rr]), sm.y);
             }
           } else {
 #pragma unroll
@@ -311,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                   while (t >= sm_bs[cb + 1]) ++cb;
                   nb = sm_bs[cb + 1];
                   sm = meta_of(cb);
+                  set_consts(sm.x);
                 }
                 const uint32_t q = (wv[jt / CPW] >> ((jt % CPW) * BITS)) & MASK;
                 v = __fmaf_rn(small_uint_to_float(q), sm.x, sm.y);
@@ -338,126 +399,145 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < C::GC; ++c) {
             uint32_t pk[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              pk[i] = (QK_F16 && tensor == 0) ? pack_f16x2(x[c * 8 + 2 * i], x[c * 8 + 2 * i + 1])
-                                              : pack_bf16x2(x[c * 8 + 2 * i], x[c * 8 + 2 * i + 1]);
+            for (int k = 0; k < 4; ++k)
+              pk[k] = (QK_F16 && tensor == 0) ? pack_f16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1])
+                                              : pack_bf16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1]);
             const int tt = g * C::GT + c * 8;  // token within the tile
             const uint32_t off = (tt >> 6) * (D * 128) + ((((tt >> 3) & 7) ^ (d & 7)) << 4);
             *reinterpret_cast<uint4*>(dst + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
         fence_async_smem();
-        mbar_arrive(tensor == 0 ? &bars->kready[ks] : &bars->vready);
+        mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
       }
-      if (*abort_flag) break;
+      if (!ok || *abort_flag) break;
       mbar_arrive(&bars->empty[st]);
-      blk = blk_lo;
     }
-  } else {
+  } else if ((warp >> 2) < NQ) {
     // ------------------------------------------------------------- softmax
-    const int r = tid;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const int i = warp >> 2;                 // query tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;    // row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
+    const uint32_t s_tmem = lane_base + col_s(i);
+    const uint32_t o_tmem = lane_base + col_o<NQ>(i);
     const float sl2 = a.scale_log2;
     float m_run = -__int_as_float(0x7F800000);
     float l_run = 0.0f;
-    uint8_t* pbuf = smem + C::OFF_P;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int sbuf = j & 1;
-      const uint32_t s_tmem = lane_base + (sbuf ? kColS1 : kColS0);
-      ok = wait_all(&bars->s_full[sbuf], (j >> 1) & 1, abort_flag);
+      ok = wait_all(&bars->s_full[i], j & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const int valid = min(C::NKV, t_att - j * C::NKV);
-      // pass 1: row maximum of the scaled scores.  Columns are read 32 at a
-      // time; when NKV % 32 == 16 the last read re-covers 16 columns.
+      // pass 1: row maximum of the raw scores
       float mx = -__int_as_float(0x7F800000);
 #pragma unroll
       for (int c0 = 0; c0 < C::NKV; c0 += 32) {
-        const int lo = (c0 + 32 <= C::NKV) ? c0 : C::NKV - 32;
-        uint32_t v[32];
-        tmem_ld32(s_tmem + lo, v);
-        tmem_wait_ld_dep(v);
+        if (c0 + 32 <= C::NKV) {
+          uint32_t v[32];
+          tmem_ld32(s_tmem + c0, v);
+          tmem_wait_ld_dep(v);
+          if (valid == C::NKV) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (lo + i >= c0 && lo + i < valid) mx = fmaxf(mx, __uint_as_float(v[i]));
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(v[k]));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (c0 + k < valid) mx = fmaxf(mx, __uint_as_float(v[k]));
+          }
+        } else {
+          uint32_t v[16];
+          tmem_ld16(s_tmem + c0, v);
+          tmem_wait_ld_dep16(v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (c0 + k < valid) mx = fmaxf(mx, __uint_as_float(v[k]));
+        }
       }
       mx *= sl2;
       float m_new = m_run;
-      if (mx > m_run + kRescaleThreshold || j == 0) m_new = fmaxf(mx, m_run);
+      if (j == 0 || mx > m_run + kRescaleThreshold) m_new = fmaxf(mx, m_run);
       const float alpha = (j == 0) ? 0.0f : ex2_approx(m_run - m_new);
-      // PV of the previous tile must be finished before O or P are touched
+      // PV_i of the previous tile has finished before O_i is rescaled
       if (j >= 1) {
-        ok = wait_all(&bars->o_done, (j - 1) & 1, abort_flag);
+        ok = wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xFFFFFFFFu, m_new != m_run)) {
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t v[32];
-            tmem_ld32(lane_base + kColO + c0, v);
+            tmem_ld32(o_tmem + c0, v);
             tmem_wait_ld_dep(v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st32(lane_base + kColO + c0, v);
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st32(o_tmem + c0, v);
           }
-          tmem_wait_st();
         }
       }
-      // pass 2: P = exp2(S * scale_log2 - m_new) as bf16 into the P tile
+      // pass 2: P = exp2(S * scale_log2 - m_new) as bf16 pairs over the consumed S columns
+      const float neg_m = -m_new;
       float rs = 0.0f;
 #pragma unroll
       for (int c0 = 0; c0 < C::NKV; c0 += 32) {
-        uint32_t v[32];
-        const int lo = (c0 + 32 <= C::NKV) ? c0 : C::NKV - 32;  // NKV % 32 == 16: reload the tail
-        tmem_ld32(s_tmem + lo, v);
-        tmem_wait_ld_dep(v);
-        float p[32];
+        if (c0 + 32 <= C::NKV) {
+          uint32_t v[32];
+          tmem_ld32(s_tmem + c0, v);
+          tmem_wait_ld_dep(v);
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = lo + i;
-          const float e = ex2_approx(__fmaf_rn(__uint_as_float(v[i]), sl2, -m_new));
-          p[i] = (col < valid) ? e : 0.0f;
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int col = lo + cc * 8;
-          if (col < c0) continue;  // tail overlap already written
-          uint32_t pk[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float p0 = p[cc * 8 + 2 * i], p1 = p[cc * 8 + 2 * i + 1];
+          for (int k = 0; k < 16; ++k) {
+            float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
+            float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
+            if (valid != C::NKV) {
+              p0 = (c0 + 2 * k < valid) ? p0 : 0.0f;
+              p1 = (c0 + 2 * k + 1 < valid) ? p1 : 0.0f;
+            }
             rs += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            pk[k] = pack_bf16x2(p0, p1);
           }
-          *reinterpret_cast<uint4*>(pbuf + sw128_offset(r, col, BM)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          tmem_st16(s_tmem + c0 / 2, pk);
+        } else {
+          uint32_t v[16];
+          tmem_ld16(s_tmem + c0, v);
+          tmem_wait_ld_dep16(v);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
+            float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
+            p0 = (c0 + 2 * k < valid) ? p0 : 0.0f;
+            p1 = (c0 + 2 * k + 1 < valid) ? p1 : 0.0f;
+            rs += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st8(s_tmem + c0 / 2, pk);
         }
       }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->s_free[sbuf]);
-      fence_async_smem();
-      mbar_arrive(&bars->p_ready);
+      mbar_arrive(&bars->p_ready[i]);
       l_run = l_run * alpha + rs;
       m_run = m_new;
     }
     // ------------------------------------------------------------- epilogue
-    if (ok && ntiles > 0 && wait_all(&bars->o_done, (ntiles - 1) & 1, abort_flag)) {
+    if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag)) {
       tc_fence_after();
-      const int row = qtile * BM + r;
+      const int row = qblk * (NQ * BM) + i * BM + r;
       const float inv = 1.0f / l_run;
       __nv_bfloat16* og = a.out + int64_t(b) * a.o_sb + int64_t(h) * a.o_sh + int64_t(row) * a.o_st;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(lane_base + kColO + c0, v);
+        tmem_ld32(o_tmem + c0, v);
         tmem_wait_ld_dep(v);
         if (row < a.lq) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v[c * 8 + 2 * i]) * inv, __uint_as_float(v[c * 8 + 2 * i + 1]) * inv);
+            for (int k = 0; k < 4; ++k)
+              pk[k] = pack_bf16x2(__uint_as_float(v[c * 8 + 2 * k]) * inv, __uint_as_float(v[c * 8 + 2 * k + 1]) * inv);
             *reinterpret_cast<uint4*>(og + c0 + c * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
@@ -472,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
   if (tid == 0 && bars->abort_flag) report(a.dev_status, VARQ_DEV_TIMEOUT);
 }
@@ -481,22 +561,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
 namespace {
 
-template <int BITS, int D, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE>
 cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
-  using C = Cfg<BITS, D>;
-  auto kern = attn_tc_kernel<BITS, D, ROPE>;
+  using C = Cfg<BITS, D, NQ>;
+  auto kern = attn_tc_kernel<BITS, D, NQ, ROPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.lq + BM - 1) / BM, a.heads, a.batch);
+  dim3 grid((a.lq + NQ * BM - 1) / (NQ * BM), a.heads, a.batch);
   kern<<<grid, kThreads, C::SMEM, stream>>>(a);
   return cudaGetLastError();
 }
 
+// Two query tiles per CTA when that still gives about two waves of CTAs.
+bool two_tiles(const AttnArgs& a) {
+  const int64_t ctas = int64_t((a.lq + 2 * BM - 1) / (2 * BM)) * a.heads * a.batch;
+  return a.lq > BM && ctas >= 2 * 148;
+}
+
+template <int BITS, int D>
+cudaError_t launch_d(const AttnArgs& a, cudaStream_t s) {
+  const bool rope = a.rope_cos != nullptr;
+  if (two_tiles(a)) return rope ? launch_tc<BITS, D, 2, true>(a, s) : launch_tc<BITS, D, 2, false>(a, s);
+  return rope ? launch_tc<BITS, D, 1, true>(a, s) : launch_tc<BITS, D, 1, false>(a, s);
+}
+
 template <int BITS>
 cudaError_t launch_bits(const AttnArgs& a, cudaStream_t s) {
-  const bool rope = a.rope_cos != nullptr;
-  if (a.head_dim == 128) return rope ? launch_tc<BITS, 128, true>(a, s) : launch_tc<BITS, 128, false>(a, s);
-  return rope ? launch_tc<BITS, 64, true>(a, s) : launch_tc<BITS, 64, false>(a, s);
+  return a.head_dim == 128 ? launch_d<BITS, 128>(a, s) : launch_d<BITS, 64>(a, s);
 }
 
 }  // namespace

@@ -218,3 +218,21 @@ def test_attention_full_size(name, bits, lq, _):
         rows = _sample_rows(lq, rng, n_rows)
         ref, ref_lse = _oracle_attention(k, v, q, bs, bits, w.n_blocks, b, h, rows, cos=cos_c, sin=sin_c)
         _check(out, lse, ref, ref_lse, b, h, rows)
+
+
+@pytest.mark.parametrize("D,bits,rope", [(128, 4, False), (128, 2, False), (128, 3, False), (128, 8, False),
+                                         (128, 5, False), (64, 4, False), (64, 3, False), (128, 4, True),
+                                         (64, 2, True)])
+def test_attention_two_query_tiles(D, bits, rope):
+    """Shapes with enough (batch, head) pairs that each CTA takes two 128-row
+    query tiles (lq > 128 and >= 296 CTAs), with a ragged last tile."""
+    B, H, lq = 4, 37, 300
+    sizes = [1, 4, 16, 36, 64, 144, 100]
+    bs = synth.block_starts(sizes)
+    k, v, q, cos, sin = _inputs(B, H, D, sizes, lq, seed=bits * 3 + D, rope=rope)
+    L = V.varq_cache_alloc(B, H, D, bits, bs)
+    out, lse = _gpu_attention(L, k, v, q, len(sizes), cos=cos, sin=sin, path=V.PATH_TENSOR)
+    rows = np.arange(lq)
+    for (b, h) in [(0, 0), (1, 17), (3, 36), (2, 5)]:
+        ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), b, h, rows, cos=cos, sin=sin)
+        _check(out, lse, ref, ref_lse, b, h, rows)
