@@ -22,19 +22,14 @@ struct QuantArgs {
   int64_t words_per_row;
   int32_t batch, heads, head_dim, bits, n_blocks_total, n_tokens;
   int32_t first_block, n_blocks;
-  int32_t staged;          // 1: slices staged in shared memory
+  int32_t n_list;          // blocks handled by one launch (set per launch)
+  int32_t list[VARQ_MAX_BLOCKS];
   int32_t block_start[VARQ_MAX_BLOCKS + 1];
 };
 
-struct QuantPlan {
-  int group;     // channels per work item (64, 32 or 16)
-  int cluster;   // CTAs per work item (1..8), one token slice each
-  size_t smem;   // dynamic shared memory per CTA
-  int staged;
-};
-
-QuantPlan plan_quant_pack(int head_dim, int bits, int max_block_len);
-cudaError_t launch_quant_pack(const QuantArgs& a, const QuantPlan& p, cudaStream_t stream);
+// Launches quantize+pack for blocks [first_block, first_block + n_blocks):
+// one launch for the short blocks (staged) and one for the long blocks.
+cudaError_t launch_quant_pack(const QuantArgs& a, cudaStream_t stream);
 
 // --------------------------------------------------------- unpack+dequant
 

@@ -6,33 +6,42 @@
 // retrieval" (low-bit values packed into INT32 storage); README,
 // "Memory-Efficient Runtime" (compact per-group metadata).
 //
-// Work item: one (b, h, block k, group of G channels) cell group.  A thread
-// block cluster of C CTAs shares the item: CTA r takes a word-aligned slice
-// of the block's tokens, stages it in shared memory while reducing per-channel
-// min/max (warp shuffles, then a shared-memory tree, then DSMEM across the
-// cluster), and quantizes its slice from shared memory.  The bf16 cache is
-// therefore read from HBM once.  Slices too large for shared memory are
-// re-read from global memory in the second pass instead (L2-resident in
-// practice).
+// Work item: one (b, h, block k, group of G channels) cell group, owned by
+// one CTA: no cross-CTA reduction is needed, so a CTA pays its fixed costs
+// (block-wide min/max reduction, cell constants) once per cell group.
+//   - Blocks of at most kStageRows tokens: G = 64 (128-byte row pieces).  The
+//     block is staged in shared memory while its min/max is reduced, and the
+//     codes are computed from shared memory.
+//   - Longer blocks: G = 16 (32-byte row pieces, one DRAM sector).  The first
+//     pass streams the rows from HBM (eight 16-byte loads in flight per thread)
+//     reducing min/max; the second pass re-reads the same rows, which the few
+//     hundred resident CTAs' footprints (<= ~150 KB each) keep in the 126 MB L2.
+// Min/max are reduced on packed bf16x2 with NaN-propagating instructions,
+// then with warp shuffles over the lanes that hold the same channels, then a
+// shared-memory tree across warps.
 //
 // Arithmetic is the exact fp32 definition:
 //   s = fp32(fp32(max - min) / (2^b - 1)),  q = rint(fp32(fp32(x - min) / s)).
-// The quotient is formed as y = (x - min) * fp32(1/s); wherever y lies within
-// 2^-13 of a half-integer the true IEEE quotient __fdiv_rn decides instead.
-// Away from those points y and the correctly rounded quotient differ by less
-// than 3 * 2^-24 * |y| < 2^-13 (|y| < 2^8), so both round to the same integer.
-#include <cooperative_groups.h>
+// Fast path: y = fma(x, fp32(1/s), -fp32(min/s)) and q = rint(y) via the
+// 1.5*2^23 rounding constant.  y differs from the correctly rounded quotient
+// by less than delta = 2^-21 (2|min/s| + 2^b + 2) (a few fp32 roundings of
+// terms bounded by |min/s| and 2^b), so wherever y lies farther than delta
+// from a half-integer both round to the same integer.  The fast path is
+// branch-free; a code inside that window (or with a non-finite y) is marked
+// and recomputed alone with __fdiv_rn afterwards.
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace varq {
 
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 8;          // rows per thread loaded back to back
+constexpr int kStageRows = 256;    // blocks up to this length are staged in shared memory
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer (ties to even)
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
@@ -44,130 +53,85 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
-__device__ __forceinline__ bool any_nonfinite_bf16x8(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    bad |= (w[i] & 0x7F80u) == 0x7F80u;
-    bad |= (w[i] & 0x7F800000u) == 0x7F800000u;
-  }
-  return bad;
-}
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) { return *reinterpret_cast<__nv_bfloat162*>(&w); }
 
-// Code of one value: q = rint((x - m) / s) clamped to [0, qmax]; 0 if s == 0.
+// Exact code of one value (the definition; used off the fast path).
 template <int BITS>
-__device__ __forceinline__ uint32_t quant_code(float x, float m, float s, float r) {
-  constexpr uint32_t qmax = (1u << BITS) - 1u;
-  const float d = __fsub_rn(x, m);
-  float y = __fmul_rn(d, r);
-  float yq = __fadd_rn(y, kMagic);
-  const float qf = __fsub_rn(yq, kMagic);
-  // within 2^-13 of a tie, or not finite (s subnormal): the IEEE quotient decides
-  if (!(fabsf(__fsub_rn(y, qf)) <= 0.5f - 1.220703125e-4f)) {
-    y = __fdiv_rn(d, s);
-    yq = __fadd_rn(y, kMagic);
-  }
-  uint32_t q = __float_as_uint(yq) & 0x3FFFFFu;
-  q = min(q, qmax);
-  return s == 0.0f ? 0u : q;
+__device__ __forceinline__ uint32_t exact_code(float x, float m, float s) {
+  if (s == 0.0f) return 0u;
+  const float y = rintf(__fdiv_rn(__fsub_rn(x, m), s));
+  const float c = fminf(fmaxf(y, 0.0f), float((1u << BITS) - 1u));
+  return static_cast<uint32_t>(c);
 }
 
-}  // namespace
+// One work item: a whole block of one (b, h) for G channels.
+struct Item {
+  int b, h, g, k;
+  int t0, t1;                 // the block's tokens
+  const __nv_bfloat16* xg;    // token t0, channel g*G of (b, h)
+};
 
-template <int BITS, int G>
-__global__ void __launch_bounds__(kThreads)
-    quant_pack_kernel(const __grid_constant__ QuantArgs a) {
-  constexpr int CPW = 32 / BITS;
-  constexpr int TPR = G / 8;             // threads per token row (8 channels each)
-  constexpr int RPI = kThreads / TPR;    // rows (or words) per pass over the CTA
-  constexpr float QMAX = float((1u << BITS) - 1u);
-  constexpr uint32_t USED = uint32_t(CPW * BITS) == 32u ? 0xFFFFFFFFu : ((1u << (CPW * BITS)) - 1u);
-
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ float red_mn[kThreads / 32][G];
-  __shared__ float red_mx[kThreads / 32][G];
-  __shared__ float part_mn[G], part_mx[G];
-  __shared__ float cell_s[G], cell_r[G], cell_m[G];
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int rank = static_cast<int>(cluster.block_rank());
-
+template <int G>
+__device__ __forceinline__ Item decode(const QuantArgs& a, int64_t item) {
+  Item it;
   const int groups = a.head_dim / G;
-  const int64_t item = static_cast<int64_t>(blockIdx.x) / C;
-  const int g = static_cast<int>(item % groups);
+  const int64_t bhn = int64_t(a.batch) * a.heads;
+  it.g = static_cast<int>(item % groups);
   const int64_t rest = item / groups;
-  const int bh = static_cast<int>(rest % (int64_t(a.batch) * a.heads));
-  const int k = a.first_block + static_cast<int>(rest / (int64_t(a.batch) * a.heads));
-  const int b = bh / a.heads, h = bh % a.heads;
+  const int bh = static_cast<int>(rest % bhn);
+  it.k = a.list[rest / bhn];
+  it.b = bh / a.heads;
+  it.h = bh % a.heads;
+  it.t0 = a.block_start[it.k];
+  it.t1 = a.block_start[it.k + 1];
+  it.xg = a.x + int64_t(it.b) * a.sb + int64_t(it.h) * a.sh + int64_t(it.t0 - a.block_start[a.first_block]) * a.st +
+          it.g * G;
+  return it;
+}
 
-  const int t0 = a.block_start[k], t1 = a.block_start[k + 1];
-  const int len = t1 - t0;
-  const int per = (len + C - 1) / C;
-  auto bound = [&](int r) -> int {
-    if (r <= 0) return t0;
-    if (r >= C) return t1;
-    int v = t0 + r * per;
-    v = ((v + CPW - 1) / CPW) * CPW;
-    return v < t0 ? t0 : (v > t1 ? t1 : v);
-  };
-  const int sa = bound(rank), sb_ = bound(rank + 1);  // this CTA's token slice [sa, sb_)
-  const int rows = sb_ - sa;
+struct Partial {
+  __nv_bfloat162 mn2[4], mx2[4];
+  bool seen;
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mn2[i] = as_bf2(0x7F807F80u);
+      mx2[i] = as_bf2(0xFF80FF80u);
+    }
+    seen = false;
+  }
+  __device__ __forceinline__ void add(const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mn2[i] = __hmin2_nan(mn2[i], as_bf2(w[i]));
+      mx2[i] = __hmax2_nan(mx2[i], as_bf2(w[i]));
+    }
+    seen = true;
+  }
+};
 
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int oct = tid % TPR;      // channel octet within the group
-  const int c8 = oct * 8;
-  const int sub = tid / TPR;      // row / word index within one pass
-
-  const __nv_bfloat16* xg = a.x + int64_t(b) * a.sb + int64_t(h) * a.sh +
-                            int64_t(t0 - a.block_start[a.first_block]) * a.st + g * G + c8;
-  uint4* stage = reinterpret_cast<uint4*>(smem_raw);  // [rows][G/8] uint4 when staged
-  const bool staged = a.staged != 0;
-
-  // ---- pass 1: min / max over the slice (and staging) ----
+// Per-thread partials -> per-channel min/max of the block (threads tid < G
+// receive channel tid).  Returns whether any input was NaN or infinite.
+template <int G>
+__device__ __forceinline__ bool block_reduce(Partial& p, float (*red_mn)[G], float (*red_mx)[G], float& out_mn,
+                                             float& out_mx) {
+  constexpr int TPR = G / 8;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c8 = (tid % TPR) * 8;
   float mn[8], mx[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    mn[i] = __int_as_float(0x7F800000);
-    mx[i] = -__int_as_float(0x7F800000);
+  for (int i = 0; i < 4; ++i) {
+    mn[2 * i] = __low2float(p.mn2[i]);
+    mn[2 * i + 1] = __high2float(p.mn2[i]);
+    mx[2 * i] = __low2float(p.mx2[i]);
+    mx[2 * i + 1] = __high2float(p.mx2[i]);
   }
+  // a NaN or infinite input shows in this thread's NaN-propagating min/max
   bool bad = false;
-  {
-    int r = sub;
-    for (; r + 3 * RPI < rows; r += 4 * RPI) {
-      uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = __ldg(reinterpret_cast<const uint4*>(xg + int64_t(sa - t0 + r + u * RPI) * a.st));
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (staged) stage[(r + u * RPI) * TPR + oct] = v[u];
-        bad |= any_nonfinite_bf16x8(v[u]);
-        float f[8];
-        bf16x8_to_f32(v[u], f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          mn[i] = fminf(mn[i], f[i]);
-          mx[i] = fmaxf(mx[i], f[i]);
-        }
-      }
-    }
-    for (; r < rows; r += RPI) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(xg + int64_t(sa - t0 + r) * a.st));
-      if (staged) stage[r * TPR + oct] = v;
-      bad |= any_nonfinite_bf16x8(v);
-      float f[8];
-      bf16x8_to_f32(v, f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        mn[i] = fminf(mn[i], f[i]);
-        mx[i] = fmaxf(mx[i], f[i]);
-      }
-    }
-  }
-  // lanes with equal `oct` hold the same channels: butterfly over the others
+  for (int i = 0; i < 8; ++i) bad |= p.seen && !(fabsf(mn[i]) <= 3.4e38f && fabsf(mx[i]) <= 3.4e38f);
+  // lanes with equal tid % TPR hold the same channels: butterfly over the others
 #pragma unroll
   for (int off = TPR; off < 32; off <<= 1) {
 #pragma unroll
@@ -183,96 +147,173 @@ __global__ void __launch_bounds__(kThreads)
       red_mx[warp][c8 + i] = mx[i];
     }
   }
-  const int any_bad = __syncthreads_or(bad ? 1 : 0);
+  const bool any_bad = __syncthreads_or(bad ? 1 : 0) != 0;
   if (tid < G) {
     float m0 = red_mn[0][tid], m1 = red_mx[0][tid];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) {
+    for (int w = 1; w < kWarps; ++w) {
       m0 = fminf(m0, red_mn[w][tid]);
       m1 = fmaxf(m1, red_mx[w][tid]);
     }
-    part_mn[tid] = m0;
-    part_mx[tid] = m1;
+    out_mn = m0;
+    out_mx = m1;
   }
-  cluster.sync();
-  // ---- cluster-wide reduction through distributed shared memory ----
-  if (tid < G) {
-    float m0 = part_mn[tid], m1 = part_mx[tid];
-    for (int r = 0; r < C; ++r) {
-      if (r == rank) continue;
-      const float* rmn = cluster.map_shared_rank(part_mn, r);
-      const float* rmx = cluster.map_shared_rank(part_mx, r);
-      m0 = fminf(m0, rmn[tid]);
-      m1 = fmaxf(m1, rmx[tid]);
-    }
-    const float s = __fdiv_rn(__fsub_rn(m1, m0), QMAX);
-    cell_s[tid] = s;
-    cell_r[tid] = s == 0.0f ? 0.0f : __frcp_rn(s);
-    cell_m[tid] = m0;
-    if (rank == 0) {
-      const uint32_t lo = __half_as_ushort(__float2half_rn(s));
-      const uint32_t hi = __half_as_ushort(__float2half_rn(m0));
-      a.meta[((int64_t(b) * a.heads + h) * a.n_blocks_total + k) * a.head_dim + g * G + tid] = lo | (hi << 16);
-      if (!(fabsf(m0) <= 65504.0f) || !(s <= 65504.0f)) report(a.dev_status, VARQ_DEV_META_OVERFLOW);
-    }
-  }
-  cluster.sync();  // partials read by every rank; cell_* visible in the CTA
-  if (any_bad && tid == 0) report(a.dev_status, VARQ_DEV_NONFINITE);
+  return any_bad;
+}
 
-  // ---- pass 2: codes, packed along tokens, CPW codes per word ----
-  float cs[8], cr[8], cm[8];
+// Cell constants and the metadata word of channel tid (thread tid < G).
+template <int BITS, int G>
+__device__ __forceinline__ void cell_constants(const QuantArgs& a, const Item& it, float m0, float m1, float* cell_s,
+                                               float* cell_r, float* cell_nmr, float* cell_m, float* cell_dl) {
+  constexpr float QMAX = float((1u << BITS) - 1u);
+  const int tid = threadIdx.x;
+  const float s = __fdiv_rn(__fsub_rn(m1, m0), QMAX);
+  const float rcp = s == 0.0f ? 0.0f : __frcp_rn(s);
+  const float mr = __fmul_rn(m0, rcp);
+  cell_s[tid] = s;
+  cell_r[tid] = rcp;
+  cell_nmr[tid] = -mr;
+  cell_m[tid] = m0;
+  cell_dl[tid] = 0.5f - (2.0f * fabsf(mr) + float(1u << BITS) + 2.0f) * 4.76837158203125e-7f;  // 0.5 - delta
+  const uint32_t lo = __half_as_ushort(__float2half_rn(s));
+  const uint32_t hi = __half_as_ushort(__float2half_rn(m0));
+  a.meta[((int64_t(it.b) * a.heads + it.h) * a.n_blocks_total + it.k) * a.head_dim + it.g * G + tid] = lo | (hi << 16);
+  if (!(fabsf(m0) <= 65504.0f) || !(s <= 65504.0f)) report(a.dev_status, VARQ_DEV_META_OVERFLOW);
+}
+
+// Second pass over one block: codes packed CPW per word, stored (words
+// shared with a neighbouring block updated atomically).  `row(t)` returns
+// channels c8..c8+7 of token t and `elem(t, i)` channel c8 + i.  The fast
+// path is branch-free so that the 8 x CPW codes of a word are independent;
+// codes near a rounding tie are marked in a bit mask and recomputed after.
+template <int BITS, int G, class RowFn, class ElemFn>
+__device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, const float* cell_s, const float* cell_r,
+                                           const float* cell_nmr, const float* cell_m, const float* cell_dl, RowFn row,
+                                           ElemFn elem) {
+  constexpr int CPW = 32 / BITS;
+  constexpr int TPR = G / 8;
+  constexpr int RPI = kThreads / TPR;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr uint32_t USED = uint32_t(CPW * BITS) == 32u ? 0xFFFFFFFFu : ((1u << (CPW * BITS)) - 1u);
+  const int tid = threadIdx.x;
+  const int c8 = (tid % TPR) * 8;
+  const int sub = tid / TPR;
+  float cr[8], cn[8], cd[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    cs[i] = cell_s[c8 + i];
     cr[i] = cell_r[c8 + i];
-    cm[i] = cell_m[c8 + i];
+    cn[i] = cell_nmr[c8 + i];
+    cd[i] = cell_dl[c8 + i];
   }
-  if (rows <= 0) return;
-  const int w_lo = sa / CPW;
-  const int w_hi = (sb_ - 1) / CPW;
-  const bool last_block = (t1 == a.n_tokens);
-  uint32_t* pk = a.packed + (int64_t(b) * a.heads + h) * a.words_per_row * a.head_dim + g * G + c8;
-
+  const int w_lo = it.t0 / CPW;
+  const int w_hi = (it.t1 - 1) / CPW;
+  const bool last_block = (it.t1 == a.n_tokens);
+  uint32_t* pk = a.packed + (int64_t(it.b) * a.heads + it.h) * a.words_per_row * a.head_dim + it.g * G + c8;
   for (int w = w_lo + sub; w <= w_hi; w += RPI) {
     const int tw = w * CPW;
-    uint32_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool full = (tw >= it.t0) && (tw + CPW <= it.t1);  // every slot in this block
+    uint32_t word[8], exc[8];
     uint32_t own = 0;
-    uint4 v[CPW];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word[i] = exc[i] = 0;
 #pragma unroll
     for (int j = 0; j < CPW; ++j) {
       const int t = tw + j;
-      const bool mine = (t >= sa) && (t < sb_);
-      v[j] = make_uint4(0, 0, 0, 0);
-      if (mine) {
-        if (staged)
-          v[j] = stage[(t - sa) * TPR + oct];
-        else
-          v[j] = __ldg(reinterpret_cast<const uint4*>(xg + int64_t(t - t0) * a.st));
+      const bool mine = full || (t >= it.t0 && t < it.t1);
+      if (mine || (last_block && t >= it.t1)) own |= MASK << (j * BITS);
+      if (!mine) continue;
+      float f[8];
+      bf16x8_to_f32(row(t), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float y = __fmaf_rn(f[i], cr[i], cn[i]);
+        const float yq = __fadd_rn(y, kMagic);
+        const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
+        // false near a tie or when y is not finite; the field is rewritten below
+        exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
+        word[i] |= (__float_as_uint(yq) & MASK) << (j * BITS);
       }
     }
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int t = tw + j;
-      const bool mine = (t >= t0) && (t < t1);
-      if (mine || (last_block && t >= t1)) own |= ((1u << BITS) - 1u) << (j * BITS);
-      if (!mine) continue;
-      float f[8];
-      bf16x8_to_f32(v[j], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] |= quant_code<BITS>(f[i], cm[i], cs[i], cr[i]) << (j * BITS);
+    for (int i = 0; i < 8; ++i) {
+      // codes near a rounding tie: the exact quotient decides
+      while (exc[i] != 0u) {
+        const int j = __ffs(exc[i]) - 1;
+        exc[i] &= exc[i] - 1u;
+        const uint32_t q = exact_code<BITS>(elem(tw + j, i), cell_m[c8 + i], cell_s[c8 + i]);
+        word[i] = (word[i] & ~(MASK << (j * BITS))) | (q << (j * BITS));
+      }
     }
-    if (tw >= t0 && tw < t1) own |= ~USED;  // unused high bits belong to slot 0's block
+    if (tw >= it.t0 && tw < it.t1) own |= ~USED;  // unused high bits belong to slot 0's block
     uint32_t* dst = pk + int64_t(w) * a.head_dim;
     if (own == 0xFFFFFFFFu) {
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(acc[0], acc[1], acc[2], acc[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(acc[4], acc[5], acc[6], acc[7]);
+      reinterpret_cast<uint4*>(dst)[0] = make_uint4(word[0], word[1], word[2], word[3]);
+      reinterpret_cast<uint4*>(dst)[1] = make_uint4(word[4], word[5], word[6], word[7]);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         atomicAnd(dst + i, ~own);
-        atomicOr(dst + i, acc[i]);
+        atomicOr(dst + i, word[i] & own);
       }
     }
+  }
+}
+
+}  // namespace
+
+// One CTA per (b, h, block, G channels).  STAGED: the block sits in shared
+// memory between the passes; otherwise the second pass re-reads it (L2).
+template <int BITS, int G, bool STAGED>
+__global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_constant__ QuantArgs a) {
+  constexpr int TPR = G / 8;
+  constexpr int RPI = kThreads / TPR;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ float red_mn[kWarps][G];
+  __shared__ float red_mx[kWarps][G];
+  __shared__ float cell_s[G], cell_r[G], cell_nmr[G], cell_m[G], cell_dl[G];
+  const int tid = threadIdx.x;
+  const int oct = tid % TPR;
+  const int c8 = oct * 8;
+  const int sub = tid / TPR;
+  const Item it = decode<G>(a, blockIdx.x);
+  const int rows = it.t1 - it.t0;
+  uint4* stage = reinterpret_cast<uint4*>(smem_raw);  // [rows][G/8] when STAGED
+
+  // ---- pass 1: min / max, kBatch 16-byte loads in flight per thread ----
+  Partial p;
+  p.init();
+  for (int base = 0; base < rows; base += RPI * kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = base + sub + u * RPI;
+      if (r < rows) v[u] = __ldg(reinterpret_cast<const uint4*>(it.xg + int64_t(r) * a.st + c8));
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = base + sub + u * RPI;
+      if (r < rows) {
+        if (STAGED) stage[r * TPR + oct] = v[u];
+        p.add(v[u]);
+      }
+    }
+  }
+  float m0 = 0.0f, m1 = 0.0f;
+  if (block_reduce<G>(p, red_mn, red_mx, m0, m1) && tid == 0) report(a.dev_status, VARQ_DEV_NONFINITE);
+  if (tid < G) cell_constants<BITS, G>(a, it, m0, m1, cell_s, cell_r, cell_nmr, cell_m, cell_dl);
+  __syncthreads();
+
+  // ---- pass 2: codes ----
+  if (STAGED) {
+    const __nv_bfloat16* st16 = reinterpret_cast<const __nv_bfloat16*>(stage);
+    pack_block<BITS, G>(
+        a, it, cell_s, cell_r, cell_nmr, cell_m, cell_dl, [&](int t) { return stage[(t - it.t0) * TPR + oct]; },
+        [&](int t, int i) { return __bfloat162float(st16[(t - it.t0) * G + c8 + i]); });
+  } else {
+    pack_block<BITS, G>(
+        a, it, cell_s, cell_r, cell_nmr, cell_m, cell_dl,
+        [&](int t) { return __ldg(reinterpret_cast<const uint4*>(it.xg + int64_t(t - it.t0) * a.st + c8)); },
+        [&](int t, int i) { return __bfloat162float(it.xg[int64_t(t - it.t0) * a.st + c8 + i]); });
   }
 }
 
@@ -280,66 +321,55 @@ __global__ void __launch_bounds__(kThreads)
 
 namespace {
 
-template <int BITS, int G>
-cudaError_t launch_qp(const QuantArgs& a, int cluster, size_t smem, int64_t grid, cudaStream_t stream) {
-  auto kern = quant_pack_kernel<BITS, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+template <int BITS, int G, bool STAGED>
+cudaError_t launch_one(const QuantArgs& a, int max_len, cudaStream_t stream) {
+  auto kern = quant_pack_kernel<BITS, G, STAGED>;
+  const size_t smem = STAGED ? size_t(max_len) * G * 2 : 0;
+  if (STAGED) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t grid = int64_t(a.n_list) * a.batch * a.heads * (a.head_dim / G);
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 template <int BITS>
-cudaError_t launch_bits(const QuantArgs& a, int g, int cluster, size_t smem, int64_t grid, cudaStream_t s) {
-  switch (g) {
-    case 64: return launch_qp<BITS, 64>(a, cluster, smem, grid, s);
-    case 32: return launch_qp<BITS, 32>(a, cluster, smem, grid, s);
-    default: return launch_qp<BITS, 16>(a, cluster, smem, grid, s);
-  }
+cudaError_t launch_bits(const QuantArgs& a, bool staged, int max_len, cudaStream_t s) {
+  return staged ? launch_one<BITS, 64, true>(a, max_len, s) : launch_one<BITS, 16, false>(a, max_len, s);
 }
 
 }  // namespace
 
-QuantPlan plan_quant_pack(int head_dim, int bits, int max_block_len) {
-  // Smallest cluster, then widest channel group, whose staged slice fits.
-  constexpr size_t kSmemBudget = 96 * 1024;
-  const int cpw = 32 / bits;
-  const int gs[3] = {head_dim < 64 ? head_dim : 64, 32, 16};
-  for (int gi = 0; gi < 3; ++gi) {
-    for (int c = 1; c <= 8; c *= 2) {
-      const int rows = (max_block_len + c - 1) / c + cpw;
-      const size_t bytes = size_t(rows) * gs[gi] * 2;
-      if (bytes <= kSmemBudget) return QuantPlan{gs[gi], c, bytes, 1};
+cudaError_t launch_quant_pack(const QuantArgs& base, cudaStream_t stream) {
+  for (int pass = 0; pass < 2; ++pass) {  // 0: short blocks (staged), 1: long blocks (two-pass via L2)
+    QuantArgs a = base;
+    a.n_list = 0;
+    int max_len = 0;
+    for (int k = base.first_block; k < base.first_block + base.n_blocks; ++k) {
+      const int len = base.block_start[k + 1] - base.block_start[k];
+      if ((len <= kStageRows) != (pass == 0)) continue;
+      a.list[a.n_list++] = k;
+      max_len = std::max(max_len, len);
     }
+    if (a.n_list == 0) continue;
+    // longest blocks first: their CTAs run longest, so they start in the first wave
+    std::stable_sort(a.list, a.list + a.n_list, [&](int x, int y) {
+      return base.block_start[x + 1] - base.block_start[x] > base.block_start[y + 1] - base.block_start[y];
+    });
+    cudaError_t e;
+    switch (a.bits) {
+      case 2: e = launch_bits<2>(a, pass == 0, max_len, stream); break;
+      case 3: e = launch_bits<3>(a, pass == 0, max_len, stream); break;
+      case 4: e = launch_bits<4>(a, pass == 0, max_len, stream); break;
+      case 5: e = launch_bits<5>(a, pass == 0, max_len, stream); break;
+      case 6: e = launch_bits<6>(a, pass == 0, max_len, stream); break;
+      case 7: e = launch_bits<7>(a, pass == 0, max_len, stream); break;
+      default: e = launch_bits<8>(a, pass == 0, max_len, stream); break;
+    }
+    if (e != cudaSuccess) return e;
   }
-  return QuantPlan{gs[0], 8, 0, 0};  // huge blocks: second pass re-reads global memory
-}
-
-cudaError_t launch_quant_pack(const QuantArgs& a, const QuantPlan& p, cudaStream_t stream) {
-  const int64_t items = int64_t(a.n_blocks) * a.batch * a.heads * (a.head_dim / p.group);
-  const int64_t grid = items * p.cluster;
-  QuantArgs aa = a;
-  aa.staged = p.staged;
-  switch (a.bits) {
-    case 2: return launch_bits<2>(aa, p.group, p.cluster, p.smem, grid, stream);
-    case 3: return launch_bits<3>(aa, p.group, p.cluster, p.smem, grid, stream);
-    case 4: return launch_bits<4>(aa, p.group, p.cluster, p.smem, grid, stream);
-    case 5: return launch_bits<5>(aa, p.group, p.cluster, p.smem, grid, stream);
-    case 6: return launch_bits<6>(aa, p.group, p.cluster, p.smem, grid, stream);
-    case 7: return launch_bits<7>(aa, p.group, p.cluster, p.smem, grid, stream);
-    default: return launch_bits<8>(aa, p.group, p.cluster, p.smem, grid, stream);
-  }
+  return cudaSuccess;
 }
 
 }  // namespace varq

@@ -90,11 +90,6 @@ int varq_quantize_pack(const varq_cache_layout* L, const void* x, int64_t sb, in
   if (first_block < 0 || n_blocks < 1 || first_block + n_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(meta)) return VARQ_ERR_ALIGNMENT;
   if (!stride_ok(sb) || !stride_ok(sh) || !stride_ok(st)) return VARQ_ERR_ALIGNMENT;
-  int max_len = 0;
-  for (int k = first_block; k < first_block + n_blocks; ++k) {
-    const int len = L->block_start[k + 1] - L->block_start[k];
-    if (len > max_len) max_len = len;
-  }
   QuantArgs a;
   std::memset(&a, 0, sizeof(a));
   a.x = static_cast<const __nv_bfloat16*>(x);
@@ -114,8 +109,7 @@ int varq_quantize_pack(const varq_cache_layout* L, const void* x, int64_t sb, in
   a.first_block = first_block;
   a.n_blocks = n_blocks;
   std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
-  const varq::QuantPlan plan = varq::plan_quant_pack(L->head_dim, L->bits, max_len);
-  return launch_status(varq::launch_quant_pack(a, plan, static_cast<cudaStream_t>(stream)));
+  return launch_status(varq::launch_quant_pack(a, static_cast<cudaStream_t>(stream)));
 }
 
 int varq_unpack_dequant(const varq_cache_layout* L, const uint32_t* packed, const uint32_t* meta, int first_block,
