@@ -18,8 +18,9 @@
 //               into the 128-byte swizzled operand layout the MMA reads
 //               (optionally rotating key pairs for the pre-RoPE key mode).
 //   warp 16     producer: 1-D bulk copies (TMA engine) of the packed K/V
-//               word rows of a tile (and of metadata rows when shared
-//               memory allows), mbarrier transaction counts.
+//               word rows of a tile, mbarrier transaction counts.  Each
+//               dequant thread keeps the (scale, min) words of its channel
+//               for the current and the next block in registers.
 //   warp 17     MMA issuer: S_i = Q_i K^T into TMEM, O_i += P_i V with P read
 //               from TMEM, tcgen05.commit to mbarriers.  Issue order per KV
 //               tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so each softmax
@@ -75,27 +76,22 @@ struct Cfg {
   static constexpr uint32_t Q_BYTES = NQ * Q_TILE_BYTES;
   static constexpr uint32_t KV_BYTES = PANELS * D * 128;
   static constexpr uint32_t WORDS_BYTES = NW * D * 4;
-  static constexpr uint32_t need(int pst, int kst, int vst, int rows) {
-    return Q_BYTES + (kst + vst) * KV_BYTES + pst * (2 * WORDS_BYTES + 2 * rows * D * 4) + kBarBytes;
+  static constexpr uint32_t need(int pst, int kst, int vst) {
+    return Q_BYTES + (kst + vst) * KV_BYTES + pst * 2 * WORDS_BYTES + kBarBytes;
   }
-  // buffer counts: prefer 2 packed stages, then double-buffered K and V,
-  // then as many staged metadata rows (<= 8) as fit
+  // buffer counts: prefer 2 packed stages, then double-buffered K and V
   static constexpr int pick() {
     const int opts[5][3] = {{2, 2, 2}, {2, 2, 1}, {1, 2, 2}, {2, 1, 1}, {1, 1, 1}};
     for (int o = 0; o < 5; ++o)
-      for (int r = 8; r >= 0; --r)
-        if (need(opts[o][0], opts[o][1], opts[o][2], r) <= kSmemUsable) return o * 16 + r;
+      if (need(opts[o][0], opts[o][1], opts[o][2]) <= kSmemUsable) return o;
     return -1;
   }
-  static constexpr int PICK = pick();
-  static_assert(PICK >= 0, "shared memory budget");
-  static constexpr int OPT = PICK / 16;
+  static constexpr int OPT = pick();
+  static_assert(OPT >= 0, "shared memory budget");
   static constexpr int PST = (OPT == 2 || OPT == 4) ? 1 : 2;
   static constexpr int KST = (OPT == 3 || OPT == 4) ? 1 : 2;
   static constexpr int VST = (OPT == 0 || OPT == 2) ? 2 : 1;
-  static constexpr int META_ROWS = PICK % 16;
-  static constexpr uint32_t META_BYTES = META_ROWS * D * 4;
-  static constexpr uint32_t STAGE_BYTES = 2 * WORDS_BYTES + 2 * META_BYTES;
+  static constexpr uint32_t STAGE_BYTES = 2 * WORDS_BYTES;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
@@ -201,9 +197,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int64_t bh = int64_t(b) * a.heads + h;
       const uint32_t* kw = a.k_packed + bh * a.words_per_row * D;
       const uint32_t* vw = a.v_packed + bh * a.words_per_row * D;
-      const uint32_t* km = a.k_meta + bh * a.n_blocks_total * D;
-      const uint32_t* vm = a.v_meta + bh * a.n_blocks_total * D;
-      int blk = 0;
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % C::PST;
@@ -212,24 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int nw = min(C::NW, words_att - w0);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
         const uint32_t wbytes = uint32_t(nw) * D * 4;
-        uint32_t mbytes = 0;
-        int blk_lo = blk;
-        if (C::META_ROWS > 0) {
-          const int tok0 = w0 * CPW;
-          const int tok1 = min(tok0 + C::NKV, t_att);
-          while (tok0 >= sm_bs[blk + 1]) ++blk;
-          blk_lo = blk;
-          int blk_hi = blk;
-          while (tok1 - 1 >= sm_bs[blk_hi + 1]) ++blk_hi;
-          mbytes = uint32_t(min(blk_hi - blk_lo + 1, C::META_ROWS)) * D * 4;
-        }
-        mbar_arrive_expect_tx(&bars->full[st], 2 * wbytes + 2 * mbytes);
+        mbar_arrive_expect_tx(&bars->full[st], 2 * wbytes);
         bulk_g2s(sb, kw + int64_t(w0) * D, wbytes, &bars->full[st]);
         bulk_g2s(sb + C::WORDS_BYTES, vw + int64_t(w0) * D, wbytes, &bars->full[st]);
-        if (C::META_ROWS > 0) {
-          bulk_g2s(sb + 2 * C::WORDS_BYTES, km + int64_t(blk_lo) * D, mbytes, &bars->full[st]);
-          bulk_g2s(sb + 2 * C::WORDS_BYTES + C::META_BYTES, vm + int64_t(blk_lo) * D, mbytes, &bars->full[st]);
-        }
         issued = j + 1;
       }
       // never leave copies in flight: wait for every stage that was filled
@@ -302,14 +280,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int dt = tid - kDequantWarp0 * 32;
     const int d = dt % D;
     const int part = dt / D;
+    const int64_t bh = int64_t(b) * a.heads + h;
+    const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + d;
+    const uint32_t* mgv = a.v_meta + bh * a.n_blocks_total * D + d;
+    const int nblk = a.n_cached_blocks;
+    // (scale, min) words of this thread's channel for block blk and blk + 1,
+    // K and V, loaded one block ahead so a tile never waits on them
+    uint32_t mk_cur = __ldg(mgk), mv_cur = __ldg(mgv);
+    uint32_t mk_next = nblk > 1 ? __ldg(mgk + D) : 0u, mv_next = nblk > 1 ? __ldg(mgv + D) : 0u;
     int blk = 0;  // block of the current tile's first token (monotone)
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % C::PST;
+      const int tok0 = j * C::NKV;
+      while (tok0 >= sm_bs[blk + 1]) {
+        ++blk;
+        mk_cur = mk_next;
+        mv_cur = mv_next;
+        const bool more = blk + 1 < nblk;
+        mk_next = more ? __ldg(mgk + int64_t(blk + 1) * D) : 0u;
+        mv_next = more ? __ldg(mgv + int64_t(blk + 1) * D) : 0u;
+      }
+      const int blk_lo = blk;
       if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
       const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
-      const int tok0 = j * C::NKV;
-      while (tok0 >= sm_bs[blk + 1]) ++blk;
-      const int blk_lo = blk;
       bool ok = true;
       for (int tensor = 0; tensor < 2 && ok; ++tensor) {
         const int nbuf = tensor == 0 ? C::KST : C::VST;
@@ -320,16 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           break;
         }
         const uint32_t* words = reinterpret_cast<const uint32_t*>(sb + tensor * C::WORDS_BYTES);
-        const uint32_t* mrows =
-            reinterpret_cast<const uint32_t*>(sb + 2 * C::WORDS_BYTES + tensor * C::META_BYTES);
-        const uint32_t* mglob =
-            (tensor == 0 ? a.k_meta : a.v_meta) + (int64_t(b) * a.heads + h) * a.n_blocks_total * D + d;
         uint8_t* dst = smem + (tensor == 0 ? C::OFF_K : C::OFF_V) + buf * C::KV_BYTES + d * 128;
         int cb = blk_lo;         // current block
         int nb = sm_bs[cb + 1];  // its end
+        const uint32_t m_cur = tensor == 0 ? mk_cur : mv_cur;
+        const uint32_t m_next = tensor == 0 ? mk_next : mv_next;
+        const uint32_t* m_glob = tensor == 0 ? mgk : mgv;
         auto meta_of = [&](int k) -> float2 {
-          const uint32_t w =
-              (k - blk_lo < C::META_ROWS) ? mrows[(k - blk_lo) * D + d] : __ldg(mglob + int64_t(k) * D);
+          const uint32_t w = k == blk_lo ? m_cur : (k == blk_lo + 1 ? m_next : __ldg(m_glob + int64_t(k) * D));
           return meta_unpack(w);
         };
         float2 sm = meta_of(cb);
@@ -438,8 +429,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tmem_ld32(s_tmem + c0, v);
           tmem_wait_ld_dep(v);
           if (valid == C::NKV) {
+            float m2 = mx;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(v[k]));
+            for (int k = 0; k < 32; k += 4) {
+              mx = fmax3(mx, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+              m2 = fmax3(m2, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+            }
+            mx = fmaxf(mx, m2);
           } else {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
@@ -477,6 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       // pass 2: P = exp2(S * scale_log2 - m_new) as bf16 pairs over the consumed S columns
       const float neg_m = -m_new;
+      const uint64_t sl2p = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+      uint64_t rs2 = f2_pack(0.0f, 0.0f);
       float rs = 0.0f;
 #pragma unroll
       for (int c0 = 0; c0 < C::NKV; c0 += 32) {
@@ -485,16 +483,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tmem_ld32(s_tmem + c0, v);
           tmem_wait_ld_dep(v);
           uint32_t pk[16];
+          if (valid == C::NKV) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
-            float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
-            if (valid != C::NKV) {
+            for (int k = 0; k < 16; ++k) {
+              float t0, t1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), sl2p, negm2), t0,
+                        t1);
+              const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+              rs2 = f2_add(rs2, f2_pack(p0, p1));
+              pk[k] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
+              float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
               p0 = (c0 + 2 * k < valid) ? p0 : 0.0f;
               p1 = (c0 + 2 * k + 1 < valid) ? p1 : 0.0f;
+              rs += p0 + p1;
+              pk[k] = pack_bf16x2(p0, p1);
             }
-            rs += p0 + p1;
-            pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_tmem + c0 / 2, pk);
         } else {
@@ -517,6 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_ready[i]);
+      {
+        float r0, r1;
+        f2_unpack(rs2, r0, r1);
+        rs += r0 + r1;
+      }
       l_run = l_run * alpha + rs;
       m_run = m_new;
     }
