@@ -220,24 +220,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       constexpr uint32_t idesc_qk =
           QK_F16 ? idesc_f16_f32(BM, C::NKV, false, true) : idesc_bf16_f32(BM, C::NKV, false, true);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, false);
-      const uint32_t q_base = smem_u32(smem + C::OFF_Q);
-      const uint32_t k_base = smem_u32(smem + C::OFF_K);
-      const uint32_t v_base = smem_u32(smem + C::OFF_V);
+      // Descriptors are built once; the start-address field (bits [0,14),
+      // address / 16) of a later operand slice is the base's plus the slice
+      // offset / 16, which never carries out of the field (shared memory is
+      // below 256 KB), so each MMA costs one add per descriptor.
+      const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(smem_u32(smem + C::OFF_K), D * 128, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + C::OFF_V), 16, 1024);
       auto issue_qk = [&](int i, int j) {
-        const uint32_t kb = k_base + (j % C::KST) * C::KV_BYTES;
+        const uint64_t kd = k_desc + uint64_t(((j % C::KST) * C::KV_BYTES) >> 4);
+        const uint64_t qd = q_desc + uint64_t((i * C::Q_TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad =
-              smem_desc_sw128(q_base + i * C::Q_TILE_BYTES + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(kb + kk * 2048, D * 128, 1024);
+          const uint64_t ad = qd + uint64_t(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+          const uint64_t bd = kd + uint64_t((kk * 2048) >> 4);
           mma_ss(tmem + col_s(i), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int j) {
-        const uint32_t vb = v_base + (j % C::VST) * C::KV_BYTES;
+        const uint64_t vd = v_desc + uint64_t(((j % C::VST) * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::NKV / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = vd + uint64_t(((kk >> 2) * (D * 128) + (kk & 3) * 32) >> 4);
           mma_ts(tmem + col_o<NQ>(i), tmem + col_s(i) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };

@@ -216,27 +216,68 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
     uint32_t own = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) word[i] = exc[i] = 0;
+    if (full) {
+      // the common case: every row of the word first (loads in flight
+      // together), then the codes.  yq = 1.5 2^23 + q holds q in its low
+      // bits, so the word is sum_j bits(yq_j) 2^(j b) minus the constant
+      // sum_j bits(1.5 2^23) 2^(j b): one integer multiply-add per code.
+      own = 0xFFFFFFFFu;
+      constexpr int CH = CPW > 4 ? 4 : CPW;  // rows loaded together
 #pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int t = tw + j;
-      const bool mine = full || (t >= it.t0 && t < it.t1);
-      if (mine || (last_block && t >= it.t1)) own |= MASK << (j * BITS);
-      if (!mine) continue;
-      float f[8];
-      bf16x8_to_f32(row(t), f);
+      for (int j0 = 0; j0 < CPW; j0 += CH) {
+        uint4 v[CH];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float y = __fmaf_rn(f[i], cr[i], cn[i]);
-        const float yq = __fadd_rn(y, kMagic);
-        const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
-        // false near a tie or when y is not finite; the field is rewritten below
-        exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
-        word[i] |= (__float_as_uint(yq) & MASK) << (j * BITS);
+        for (int u = 0; u < CH; ++u)
+          if (j0 + u < CPW) v[u] = row(tw + j0 + u);
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int j = j0 + u;
+          if (j >= CPW) break;
+          float f[8];
+          bf16x8_to_f32(v[u], f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float y = __fmaf_rn(f[i], cr[i], cn[i]);
+            const float yq = __fadd_rn(y, kMagic);
+            const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
+            // false near a tie or when y is not finite; the field is rewritten below
+            exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
+            word[i] += __float_as_uint(yq) << (j * BITS);
+          }
+        }
+      }
+      constexpr uint32_t kMagicSum = [] {
+        uint32_t k = 0;
+        for (int j = 0; j < CPW; ++j) k += 0x4B400000u << (j * BITS);
+        return k;
+      }();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word[i] -= kMagicSum;
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPW; ++j) {
+        const int t = tw + j;
+        const bool mine = t >= it.t0 && t < it.t1;
+        if (mine || (last_block && t >= it.t1)) own |= MASK << (j * BITS);
+        if (!mine) continue;
+        float f[8];
+        bf16x8_to_f32(row(t), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float y = __fmaf_rn(f[i], cr[i], cn[i]);
+          const float yq = __fadd_rn(y, kMagic);
+          const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
+          exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
+          word[i] |= (__float_as_uint(yq) & MASK) << (j * BITS);
+        }
       }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      // codes near a rounding tie: the exact quotient decides
+      // codes near a rounding tie: the exact quotient decides.  (A cell with
+      // a non-finite y has every code of the word marked; the sum above may
+      // then have carried into the unused high bits, which are cleared.)
+      if (exc[i] != 0u) word[i] &= USED;
       while (exc[i] != 0u) {
         const int j = __ffs(exc[i]) - 1;
         exc[i] &= exc[i] - 1u;
