@@ -152,6 +152,15 @@ VARQ_API int varq_quantize_pack(const varq_cache_layout* layout, const void* x,
                        uint32_t* dev_status, void* stream);
 
 /*
+ * varq_quantize_pack_launches -- how many kernel launches varq_quantize_pack
+ * queues for blocks [first_block, first_block + n_blocks) of this layout (1
+ * or 2: one per group of blocks of similar length), for callers that count
+ * launches (CUDA-graph capture, profiling).  Negative varq_status on a bad
+ * layout or range.  Host only; nothing is launched.
+ */
+VARQ_API int varq_quantize_pack_launches(const varq_cache_layout* layout, int first_block, int n_blocks);
+
+/*
  * varq_unpack_dequant -- standalone unpack + dequantize of blocks
  * [first_block, first_block + n_blocks) to dense bf16 (the unfused path:
  * [PAGE] "Quantization, bit packing, and retrieval"; [README] CUDA

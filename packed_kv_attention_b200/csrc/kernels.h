@@ -30,6 +30,8 @@ struct QuantArgs {
 // Launches quantize+pack for blocks [first_block, first_block + n_blocks):
 // one launch for the short blocks (staged) and one for the long blocks.
 cudaError_t launch_quant_pack(const QuantArgs& a, cudaStream_t stream);
+// Number of kernel launches launch_quant_pack makes for these blocks.
+int quant_pack_launch_count(const QuantArgs& a);
 
 // --------------------------------------------------------- unpack+dequant
 

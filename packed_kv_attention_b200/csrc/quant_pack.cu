@@ -382,6 +382,13 @@ cudaError_t launch_bits(const QuantArgs& a, bool staged, int max_len, cudaStream
 
 }  // namespace
 
+int quant_pack_launch_count(const QuantArgs& a) {
+  bool any[2] = {false, false};
+  for (int k = a.first_block; k < a.first_block + a.n_blocks; ++k)
+    any[(a.block_start[k + 1] - a.block_start[k] <= kStageRows) ? 0 : 1] = true;
+  return int(any[0]) + int(any[1]);
+}
+
 cudaError_t launch_quant_pack(const QuantArgs& base, cudaStream_t stream) {
   for (int pass = 0; pass < 2; ++pass) {  // 0: short blocks (staged), 1: long blocks (two-pass via L2)
     QuantArgs a = base;

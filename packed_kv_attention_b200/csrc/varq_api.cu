@@ -112,6 +112,18 @@ int varq_quantize_pack(const varq_cache_layout* L, const void* x, int64_t sb, in
   return launch_status(varq::launch_quant_pack(a, static_cast<cudaStream_t>(stream)));
 }
 
+int varq_quantize_pack_launches(const varq_cache_layout* L, int first_block, int n_blocks) {
+  int rc = check_layout(L);
+  if (rc != VARQ_OK) return rc;
+  if (first_block < 0 || n_blocks < 1 || first_block + n_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
+  QuantArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.first_block = first_block;
+  a.n_blocks = n_blocks;
+  std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
+  return varq::quant_pack_launch_count(a);
+}
+
 int varq_unpack_dequant(const varq_cache_layout* L, const uint32_t* packed, const uint32_t* meta, int first_block,
                         int n_blocks, void* out, int64_t sb, int64_t sh, int64_t st, void* stream) {
   int rc = check_layout(L);

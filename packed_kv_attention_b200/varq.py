@@ -19,7 +19,7 @@ __all__ = [
     "varq_status_string", "varq_abi_version", "alloc_cache", "MAX_BLOCKS",
     "PATH_AUTO", "PATH_TENSOR", "PATH_SPLIT", "SPLIT_MAX_LQ",
     "DEV_NONFINITE", "DEV_META_OVERFLOW", "DEV_TIMEOUT",
-    "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "varq_quantize_pack_launches",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvarq.so")
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.varq_quantize_pack.argtypes = [ctypes.POINTER(CacheLayout), _c_p, _c_i64, _c_i64, _c_i64, _c_int, _c_int,
                                          _c_p, _c_p, _c_p, _c_p]
         L.varq_quantize_pack.restype = _c_int
+        L.varq_quantize_pack_launches.argtypes = [ctypes.POINTER(CacheLayout), _c_int, _c_int]
+        L.varq_quantize_pack_launches.restype = _c_int
         L.varq_unpack_dequant.argtypes = [ctypes.POINTER(CacheLayout), _c_p, _c_p, _c_int, _c_int, _c_p,
                                           _c_i64, _c_i64, _c_i64, _c_p]
         L.varq_unpack_dequant.restype = _c_int
@@ -158,6 +160,16 @@ def varq_quantize_pack(layout: CacheLayout, x: torch.Tensor, packed: torch.Tenso
     rc = lib().varq_quantize_pack(ctypes.byref(layout), _ptr(x), sb, sh, st, first_block, n_blocks,
                                   _ptr(packed), _ptr(meta), _ptr(dev_status), _stream(stream))
     _check(rc, "varq_quantize_pack")
+
+
+def varq_quantize_pack_launches(layout: CacheLayout, first_block: int = 0, n_blocks: Optional[int] = None) -> int:
+    """Kernel launches one varq_quantize_pack call queues for these blocks."""
+    if n_blocks is None:
+        n_blocks = layout.n_blocks - first_block
+    rc = lib().varq_quantize_pack_launches(ctypes.byref(layout), first_block, n_blocks)
+    if rc < 0:
+        _check(rc, "varq_quantize_pack_launches")
+    return rc
 
 
 def varq_unpack_dequant(layout: CacheLayout, packed: torch.Tensor, meta: torch.Tensor, out: torch.Tensor,

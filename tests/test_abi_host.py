@@ -161,3 +161,13 @@ def test_status_strings():
     for c in (OK, INVALID, UNSUPPORTED, CUDA, WORKSPACE, ALIGN):
         assert V.varq_status_string(c).startswith("VARQ_")
     assert "unknown" in V.varq_status_string(123)
+
+
+def test_quantize_pack_launch_count():
+    """One launch per group of blocks of similar length (<= 256 tokens, longer)."""
+    L = V.varq_cache_alloc(1, 1, 128, 4, [0, 1, 5, 21, 300, 1000])
+    assert V.varq_quantize_pack_launches(L) == 2
+    assert V.varq_quantize_pack_launches(L, 0, 3) == 1
+    assert V.varq_quantize_pack_launches(L, 3, 2) == 1
+    with pytest.raises(V.VarqError):
+        V.varq_quantize_pack_launches(L, 4, 2)
