@@ -316,6 +316,106 @@ def run_reference(args, w, rank, world):
     return 0
 
 
+def _event_times(fn, stream, iters):
+    """Per-iteration device times (ms) of fn() on stream, each bracketed by
+    CUDA events (every input below exceeds the 126 MB L2)."""
+    times = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return times
+
+
+def measure_rows(dev, stream, peaks, iters=5):
+    """The hot-path steps bench's main step does not time, each on the
+    workload made for it and against its own roofline:
+      a2-a5 quantize+pack and a6 unpack+dequant on the 1 GiB kernel-sweep
+            cache (bits 2, 3, 4, 8; inputs and outputs exceed L2);
+      a9    split-KV attention (Lq = 1 and 16) over the sweep cache (INT4);
+      a8    pre-RoPE keys: tensor-path attention of the Self-Forcing-like
+            next-frame layer (INT4, 4680 queries over 32,760 tokens)."""
+    from packed_kv_attention_b200 import varq as V
+    hbm = peaks["hbm_gbs"]
+    tflops_peak = peaks["bf16_tflops_sustained"]
+    rows = {}
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    w = synth.WORKLOADS["sweep"]
+    data = synth.make_inputs(w, lq=16, seed=3, device=dev)
+    k, v = data["k"], data["v"]
+    bs = data["block_start"]
+    out = torch.empty_like(k)
+    qp, ud = {}, {}
+    for bits in (2, 3, 4, 8):
+        L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, bs)
+        kp, km = V.alloc_cache(L, dev)
+        for _ in range(3):
+            V.varq_quantize_pack(L, k, kp, km, dev_status=st, stream=stream)
+        tq = statistics.median(_event_times(
+            lambda: V.varq_quantize_pack(L, k, kp, km, dev_status=st, stream=stream), stream, iters))
+        for _ in range(3):
+            V.varq_unpack_dequant(L, kp, km, out, stream=stream)
+        tu = statistics.median(_event_times(lambda: V.varq_unpack_dequant(L, kp, km, out, stream=stream), stream, iters))
+        nbytes = k.numel() * 2 + L.packed_bytes + L.meta_bytes
+        qp[f"int{bits}"] = {"us": 1e3 * tq, "GB/s": nbytes / (tq * 1e-3) / 1e9, "frac_hbm": nbytes / (tq * 1e-3) / 1e9 / hbm}
+        ud[f"int{bits}"] = {"us": 1e3 * tu, "GB/s": nbytes / (tu * 1e-3) / 1e9, "frac_hbm": nbytes / (tu * 1e-3) / 1e9 / hbm}
+        if bits == 4:
+            kp4, km4, L4 = kp, km, L
+    desc = f"sweep: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} blocks={w.n_blocks}"
+    rows["a2_a5_quant_pack"] = {"workload": desc, "bytes": "bf16 read + packed + metadata written", **qp}
+    rows["a6_unpack_dequant"] = {"workload": desc, "bytes": "packed + metadata read + bf16 written", **ud}
+
+    # a9: split-KV attention over the INT4 sweep cache (K and V share the packed words here)
+    vp4, vm4 = V.alloc_cache(L4, dev)
+    V.varq_quantize_pack(L4, v, vp4, vm4, dev_status=st, stream=stream)
+    split = {}
+    for lq in (1, 16):
+        q = data["q"][:, :, :lq].contiguous()
+        o = torch.empty_like(q)
+        ws_bytes = V.varq_packed_attention_workspace(L4, lq, w.n_blocks, V.PATH_SPLIT)
+        ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device=dev)
+
+        def run():
+            V.varq_packed_attention(L4, q, kp4, km4, vp4, vm4, o, workspace=ws, path=V.PATH_SPLIT,
+                                    dev_status=st, stream=stream)
+        for _ in range(3):
+            run()
+        t = statistics.median(_event_times(run, stream, iters))
+        nbytes = attention_bytes(L4, w, lq, False)
+        split[f"lq{lq}"] = {"us": 1e3 * t, "GB/s": nbytes / (t * 1e-3) / 1e9,
+                            "frac_hbm": nbytes / (t * 1e-3) / 1e9 / hbm}
+    rows["a9_split_kv"] = {"workload": desc + " INT4", "bound": "hbm",
+                           "bytes": "Q + O + packed K, V + metadata", **split}
+    del data, k, v, out, kp4, km4, vp4, vm4
+    torch.cuda.empty_cache()
+
+    # a8: pre-RoPE keys on the tensor path (Self-Forcing-like layer)
+    w = synth.WORKLOADS["self_forcing"]
+    pipe = Pipeline(w, 4, w.lq[-1], dev, seed=4)
+    pipe.step(stream)
+    torch.cuda.synchronize()
+
+    def attn():
+        V.varq_packed_attention(pipe.L, pipe.q, pipe.kp, pipe.km, pipe.vp, pipe.vm, pipe.out,
+                                rope_cos=pipe.cos, rope_sin=pipe.sin, workspace=pipe.ws,
+                                dev_status=st, stream=stream)
+    for _ in range(2):
+        attn()
+    t = statistics.median(_event_times(attn, stream, 3))
+    fl = attention_flops(w, w.lq[-1])
+    rows["a8_pre_rope_attention"] = {
+        "workload": f"self_forcing: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} Lq={w.lq[-1]} INT4 pre-RoPE",
+        "bound": "tensor", "ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12,
+        "frac_tensor": fl / (t * 1e-3) / 1e12 / tflops_peak}
+    rows["device_status"] = int(st.item())
+    del pipe
+    torch.cuda.empty_cache()
+    return rows
+
+
 def config_of(w, args):
     return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} "
                         f"blocks={w.n_blocks} Lq={args.lq} INT{args.bits}",
@@ -338,6 +438,7 @@ def main(argv=None):
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements (unpack, split-KV, pre-RoPE)")
     args = ap.parse_args(argv)
     w = synth.WORKLOADS[args.workload]
     if args.lq <= 0:
@@ -424,6 +525,11 @@ def main(argv=None):
         line["also"]["attention_frac_tensor"] = line["also"]["attention_TFLOP/s"] / tensor_peak
         del p2
         torch.cuda.empty_cache()
+        pipe = Pipeline(w, args.bits, args.lq, dev)
+    if not args.no_rows and world == 1:
+        del pipe
+        torch.cuda.empty_cache()
+        line["rows"] = measure_rows(dev, stream, peaks)
         pipe = Pipeline(w, args.bits, args.lq, dev)
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(pipe, max(3, args.steps // 2), 2, stream)

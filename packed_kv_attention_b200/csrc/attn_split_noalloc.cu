@@ -125,6 +125,7 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(float(L->head_dim));
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.kv_split = 1;
   a.n_splits = varq::split_kv_splits(a);
 
   // the shape must fit the fixed scratch array
@@ -134,6 +135,6 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   rc = scratch_on_current_device(&scratch);
   if (rc != VARQ_OK) return rc;
   a.workspace = scratch;
-  const cudaError_t e = varq::launch_attention_split(a, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = varq::launch_attention_tc(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VARQ_OK : VARQ_ERR_CUDA;
 }

@@ -37,6 +37,8 @@
 // One packed word holds consecutive tokens of one channel, so unpacking it
 // yields a contiguous run along a row of the K and V tiles in both GEMMs.
 // Q and K are fp16 instead of bf16 in the pre-RoPE key mode (QK_F16).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -143,11 +145,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int qblk = blockIdx.x;
+  const int nqb = (a.lq + NQ * BM - 1) / (NQ * BM);  // query-tile groups
+  const int qblk = blockIdx.x % nqb;
+  const int split = blockIdx.x / nqb;                   // KV range (split-KV form)
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int t_att = a.t_att;
-  const int ntiles = (t_att + C::NKV - 1) / C::NKV;
+  const int ntiles_all = (t_att + C::NKV - 1) / C::NKV;
+  const int per_split = a.kv_split ? (ntiles_all + a.n_splits - 1) / a.n_splits : ntiles_all;
+  const int tile0 = split * per_split;                  // first KV tile of this CTA
+  const int ntiles = max(0, min(ntiles_all, tile0 + per_split) - tile0);
   const int words_att = (t_att + CPW - 1) / CPW;
 
   // ------------------------------------------------------------- set-up
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % C::PST;
         if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, abort_flag)) break;
-        const int w0 = j * C::NW;
+        const int w0 = (tile0 + j) * C::NW;
         const int nw = min(C::NW, words_att - w0);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
         const uint32_t wbytes = uint32_t(nw) * D * 4;
@@ -245,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           mma_ts(tmem + col_o<NQ>(i), tmem + col_s(i) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars->kready[0], 0, abort_flag);
+      bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         for (int i = 0; i < NQ; ++i) {
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     int blk = 0;  // block of the current tile's first token (monotone)
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % C::PST;
-      const int tok0 = j * C::NKV;
+      const int tok0 = (tile0 + j) * C::NKV;
       while (tok0 >= sm_bs[blk + 1]) {
         ++blk;
         mk_cur = mk_next;
@@ -423,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       ok = wait_all(&bars->s_full[i], j & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-      const int valid = min(C::NKV, t_att - j * C::NKV);
+      const int valid = min(C::NKV, t_att - (tile0 + j) * C::NKV);
       // pass 1: row maximum of the raw scores
       float mx = -__int_as_float(0x7F800000);
 #pragma unroll
@@ -538,7 +545,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       m_run = m_new;
     }
     // ------------------------------------------------------------- epilogue
-    if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag)) {
+    if (a.kv_split) {
+      // split-KV form: the unnormalised partial of this KV range (O, running
+      // max m in the log2 domain, running sum l); m = -inf marks "no token"
+      const int row = qblk * (NQ * BM) + i * BM + r;
+      float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
+                  int64_t(row) * (D + 2);
+      const bool have = ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
+      if (have) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(o_tmem + c0, v);
+          tmem_wait_ld_dep(v);
+          if (row < a.lq) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              *reinterpret_cast<float2*>(ws + c0 + 2 * k) =
+                  make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+          }
+        }
+      }
+      if (row < a.lq) {
+        ws[D] = have ? m_run : -__int_as_float(0x7F800000);
+        ws[D + 1] = have ? l_run : 0.0f;
+      }
+    } else if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag)) {
       tc_fence_after();
       const int row = qblk * (NQ * BM) + i * BM + r;
       const float inv = 1.0f / l_run;
@@ -584,15 +617,31 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   auto kern = attn_tc_kernel<BITS, D, NQ, ROPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.lq + NQ * BM - 1) / (NQ * BM), a.heads, a.batch);
+  dim3 grid(unsigned((a.lq + NQ * BM - 1) / (NQ * BM) * (a.kv_split ? a.n_splits : 1)), a.heads, a.batch);
   kern<<<grid, kThreads, C::SMEM, stream>>>(a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !a.kv_split) return e;
+  return launch_attention_combine(a, stream);
 }
 
-// Two query tiles per CTA when that still gives about two waves of CTAs.
+// Two query tiles per CTA when that still gives about two waves of CTAs
+// (never in the split-KV form, whose query blocks are small).
 bool two_tiles(const AttnArgs& a) {
   const int64_t ctas = int64_t((a.lq + 2 * BM - 1) / (2 * BM)) * a.heads * a.batch;
-  return a.lq > BM && ctas >= 2 * 148;
+  return !a.kv_split && a.lq > BM && ctas >= 2 * 148;
+}
+
+// Tokens per KV tile for a bit width (Cfg<BITS, D, NQ>::NKV).
+int tile_tokens(int bits) {
+  const int cpw = 32 / bits;
+  int g = cpw, h = 16;
+  while (h != 0) {
+    const int t = g % h;
+    g = h;
+    h = t;
+  }
+  const int unit = cpw / g * 16;
+  return (128 / unit) * unit;
 }
 
 template <int BITS, int D>
@@ -608,6 +657,21 @@ cudaError_t launch_bits(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+// Split-KV form: enough CTAs for about two waves over 148 SMs (one CTA per
+// SM), each range at least four KV tiles long when the cache allows, and no
+// empty range.
+int split_kv_splits(const AttnArgs& a) {
+  const int nkv = tile_tokens(a.bits);
+  const int ntiles = (a.t_att + nkv - 1) / nkv;
+  const int64_t base = int64_t((a.lq + BM - 1) / BM) * a.heads * a.batch;
+  int64_t want = (2 * 148 + base - 1) / base;
+  want = std::min<int64_t>(want, std::max(1, ntiles / 4));
+  want = std::min<int64_t>(want, 64);
+  want = std::max<int64_t>(want, 1);
+  const int per = static_cast<int>((ntiles + want - 1) / want);
+  return (ntiles + per - 1) / per;
+}
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
   switch (a.bits) {

@@ -71,13 +71,18 @@ struct AttnArgs {
   int32_t t_att;           // attended tokens: block_start[n_cached_blocks]
   float scale_log2;        // softmax scale * log2(e)
   float scale;             // softmax scale
-  int32_t n_splits;        // split-KV only
+  int32_t kv_split;        // 1: each CTA attends to one of n_splits ranges of KV tiles and writes an
+                           // unnormalised partial (O, m, l) to the workspace; a combine kernel merges them
+  int32_t n_splits;
   int32_t block_start[VARQ_MAX_BLOCKS + 1];
 };
 
+// Tensor-core attention; with kv_split, the split-KV form plus its combine.
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
-cudaError_t launch_attention_split(const AttnArgs& a, cudaStream_t stream);
+// Number of KV ranges of the split-KV form for these arguments.
 int split_kv_splits(const AttnArgs& a);
 size_t split_kv_workspace_bytes(int batch, int heads, int lq, int head_dim, int n_splits);
+// The log-sum-exp merge of the split-KV partials into out (and lse).
+cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace varq

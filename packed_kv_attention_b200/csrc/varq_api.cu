@@ -229,12 +229,14 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p == VARQ_PATH_TENSOR) return launch_status(varq::launch_attention_tc(a, s));
 
+  // split-KV form: the tensor-core kernel over ranges of KV tiles, then the merge
+  a.kv_split = 1;
   a.n_splits = varq::split_kv_splits(a);
   const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits);
   if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
   a.workspace = static_cast<float*>(workspace);
-  return launch_status(varq::launch_attention_split(a, s));
+  return launch_status(varq::launch_attention_tc(a, s));
 }
 
 }  // extern "C"
