@@ -39,25 +39,15 @@
 // Q and K are fp16 instead of bf16 in the pre-RoPE key mode (QK_F16).
 #include <algorithm>
 
+#include "attn_tc_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
 namespace varq {
 
+using namespace tc;
+
 namespace {
-
-constexpr int kThreads = 576;
-constexpr int kDequantWarp0 = 8;
-constexpr int kDequantThreads = 256;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int BM = 128;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr uint32_t kSmemUsable = 227 * 1024 - 1024;  // minus 1 KB to align the base to 1024
-constexpr uint32_t kBarBytes = 2048;
-
-constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
-constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
 
 template <int BITS, int D, int NQ>
 struct Cfg {
@@ -103,27 +93,6 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
   static_assert(NKV % 16 == 0 && NKV <= 128, "tile shape");
 };
-
-__host__ __device__ constexpr uint32_t col_s(int i) { return uint32_t(i) * 128u; }
-template <int NQ>
-__host__ __device__ constexpr uint32_t col_o(int i) { return uint32_t(NQ) * 128u + uint32_t(i) * 128u; }
-
-struct Barriers {
-  uint64_t full[2], empty[2];     // packed stage filled by TMA / released by dequant
-  uint64_t kready[2], kfree[2];   // 16-bit K tile written / consumed by all S MMAs
-  uint64_t vready[2], vfree[2];   // 16-bit V tile written / consumed by all PV MMAs
-  uint64_t s_full[2];             // S_i of the current tile in TMEM
-  uint64_t p_ready[2];            // P_i in TMEM and O_i rescaled
-  uint64_t o_done[2];             // PV_i finished
-  uint64_t teardown;
-  uint32_t tmem_base;
-  int abort_flag;
-};
-
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait(bar, parity, abort_flag);
-  return __all_sync(0xFFFFFFFFu, ok);
-}
 
 }  // namespace
 
@@ -658,13 +627,21 @@ cudaError_t launch_bits(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// The paired-CTA kernel (attn_tc2.cu) dequantizes each KV tile once per pair
+// of query-tile groups.  It pays where the dequant is the bottleneck: the
+// pre-RoPE key mode (rotation per key element) on the tensor path.  Where the
+// per-tile chain softmax -> P V -> Q K^T is the bottleneck (no RoPE, and the
+// split-KV form with one query tile per CTA) the single-CTA kernel is faster:
+// the pair's cross-CTA signals lengthen that chain.
+bool use_pair_kernel(const AttnArgs& a) { return a.rope_cos != nullptr && !a.kv_split; }
+
 // Split-KV form: enough CTAs for about two waves over 148 SMs (one CTA per
 // SM), each range at least four KV tiles long when the cache allows, and no
 // empty range.
 int split_kv_splits(const AttnArgs& a) {
   const int nkv = tile_tokens(a.bits);
   const int ntiles = (a.t_att + nkv - 1) / nkv;
-  const int64_t base = int64_t((a.lq + BM - 1) / BM) * a.heads * a.batch;
+  const int64_t base = int64_t((a.lq + BM - 1) / BM) * a.heads * a.batch;  // single-CTA kernel
   int64_t want = (2 * 148 + base - 1) / base;
   want = std::min<int64_t>(want, std::max(1, ntiles / 4));
   want = std::min<int64_t>(want, 64);
@@ -674,6 +651,7 @@ int split_kv_splits(const AttnArgs& a) {
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream) {
+  if (use_pair_kernel(a)) return launch_attention_tc2(a, stream);
   switch (a.bits) {
     case 2: return launch_bits<2>(a, stream);
     case 3: return launch_bits<3>(a, stream);

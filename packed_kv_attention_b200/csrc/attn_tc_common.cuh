@@ -1,0 +1,46 @@
+// Definitions shared by the two tensor-core attention kernels (one CTA per
+// query-tile group in attn_tc.cu, a pair of CTAs sharing every MMA in
+// attn_tc2.cu): warp roles, tile constants, TMEM columns, mbarriers.
+#pragma once
+
+#include "common.cuh"
+
+namespace varq {
+namespace tc {
+
+constexpr int kThreads = 576;
+constexpr int kDequantWarp0 = 8;
+constexpr int kDequantThreads = 256;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int BM = 128;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kSmemUsable = 227 * 1024 - 1024;  // minus 1 KB to align the base to 1024
+constexpr uint32_t kBarBytes = 2048;
+
+constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
+constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
+
+__host__ __device__ constexpr uint32_t col_s(int i) { return uint32_t(i) * 128u; }
+template <int NQ>
+__host__ __device__ constexpr uint32_t col_o(int i) { return uint32_t(NQ) * 128u + uint32_t(i) * 128u; }
+
+struct Barriers {
+  uint64_t full[2], empty[2];     // packed stage filled by TMA / released by dequant
+  uint64_t kready[2], kfree[2];   // 16-bit K tile written / consumed by all S MMAs
+  uint64_t vready[2], vfree[2];   // 16-bit V tile written / consumed by all PV MMAs
+  uint64_t s_full[2];             // S_i of the current tile in TMEM
+  uint64_t p_ready[2];            // P_i in TMEM and O_i rescaled
+  uint64_t o_done[2];             // PV_i finished
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+}  // namespace tc
+}  // namespace varq

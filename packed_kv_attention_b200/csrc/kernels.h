@@ -78,7 +78,10 @@ struct AttnArgs {
 };
 
 // Tensor-core attention; with kv_split, the split-KV form plus its combine.
+// Pre-RoPE keys on the tensor path go to the paired-CTA kernel
+// (launch_attention_tc2), everything else to the single-CTA one.
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attention_tc2(const AttnArgs& a, cudaStream_t stream);
 // Number of KV ranges of the split-KV form for these arguments.
 int split_kv_splits(const AttnArgs& a);
 size_t split_kv_workspace_bytes(int batch, int heads, int lq, int head_dim, int n_splits);
