@@ -1,0 +1,454 @@
+// Split-KV form for short query blocks on the CUDA cores: attention straight
+// from the packed codes (README, "Fused-kernel overhead reduction": attention
+// reads the packed cache itself; project page, "Next-block prediction": every
+// query attends to the whole cache).
+//
+// With the per-(channel, block) affine code k = s c + m, a score is
+//   q . k_t = sum_d (q_d s_d,b) c_t,d + sum_d q_d m_d,b,
+// so per block the query is scaled once (q~_d = q_d s_d,b scale log2 e) and
+// the second sum is one bias per (block, query row); and the output is
+//   O_d = sum_b [ s_d,b sum_{t in b} p_t c_t,d + m_d,b sum_{t in b} p_t ].
+// No value is dequantized: every code costs an extract, a convert and one
+// FMA per query row, so the kernel streams the packed words at a rate set by
+// those instructions rather than by a 16-bit tile written to shared memory.
+//
+// Work split: CTA (KV range, query-row group, head, batch); its 8 warps take
+// steps of RPW word rows in turn, each warp keeping its own online-softmax
+// state (running max m per row, lane-partial sums l, O for the lane's
+// channels), merged across warps at the end into the split-KV partial
+// (O, m, l) that the log-sum-exp merge (attn_combine.cu) reduces over ranges.
+// Scores are in the log2 domain; the running max moves only when a step's
+// scores exceed it by more than kDecRescale, so P <= 2^kDecRescale.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace varq {
+
+namespace {
+
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr float kDecRescale = 8.0f;  // log2 units
+
+template <int BITS, int D, int QG>
+struct Dec {
+  static constexpr int CPW = 32 / BITS;                // tokens per word
+  static constexpr uint32_t MASK = (1u << BITS) - 1u;
+  static constexpr int NCG = D / 16;                   // K: 16-channel groups, one lane each
+  static constexpr int LOG_NCG = NCG == 8 ? 3 : 2;
+  static constexpr int RPW = 32 / NCG;                 // word rows per warp step
+  static constexpr int TPS = RPW * CPW;                // tokens per warp step
+  static constexpr int NV = QG * CPW;                  // K partial sums per lane: [row g][token j]
+  static constexpr int NVP = (NV + NCG - 1) / NCG * NCG;  // padded to a multiple of the lanes summed over
+  static constexpr int VPL = NVP / NCG;                // scores a lane holds after the reduction
+  static constexpr int CPL = D / 32;                   // V: channels per lane (lane + 32 k)
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(NV <= 32, "partial sums per lane");
+};
+
+// Code j of a packed word as an exact fp32 value.
+template <int BITS>
+__device__ __forceinline__ float code_f(uint32_t w, int j) {
+  return small_uint_to_float((w >> (j * BITS)) & ((1u << BITS) - 1u));
+}
+
+// fp32 rounded to the nearest bf16 (ties to even), as fp32.
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// Codes j and j + 1 of a word dequantized as fmaf(code, s, min) and rounded
+// to bf16 together (the second only when `two`).
+template <int BITS>
+__device__ __forceinline__ void dequant_pair(uint32_t w, int j, bool two, float s, float mn, float& x0, float& x1) {
+  const float a = __fmaf_rn(small_uint_to_float((w >> (j * BITS)) & ((1u << BITS) - 1u)), s, mn);
+  const float b = two ? __fmaf_rn(small_uint_to_float((w >> ((j + 1) * BITS)) & ((1u << BITS) - 1u)), s, mn) : 0.0f;
+  const uint32_t u = pack_bf16x2(a, b);
+  x0 = __uint_as_float(u << 16);
+  x1 = __uint_as_float(u & 0xFFFF0000u);
+}
+
+// Bit-reversed lane group index: the reduce-scatter below leaves lane cg with
+// the VPL consecutive partials starting at VPL * bitrev(cg).
+template <int L>
+__device__ __forceinline__ int bitrev(int x) {
+  return L == 3 ? (((x & 1) << 2) | (x & 2) | ((x >> 2) & 1)) : (((x & 1) << 1) | ((x >> 1) & 1));
+}
+
+// One level of the reduce-scatter: the first N values summed with lane ^ M,
+// the lane keeping the upper half if its bit M is set, in x[0, N / 2).
+template <int N, int M, int NVP>
+__device__ __forceinline__ void rs_level(float (&x)[NVP], int lane) {
+  constexpr int HALF = N / 2;
+  const bool up = (lane & M) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float send = up ? x[i] : x[i + HALF];
+    const float keep = up ? x[i + HALF] : x[i];
+    x[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, M);
+  }
+}
+
+// Sum the NVP partials over the NCG lanes of a word row (lanes differing in
+// the low LOG_NCG bits), halving the values each lane carries at every level.
+template <int NVP, int LOG_NCG>
+__device__ __forceinline__ void reduce_scatter(float (&x)[NVP], int lane) {
+  rs_level<NVP, 1>(x, lane);
+  rs_level<NVP / 2, 2>(x, lane);
+  if constexpr (LOG_NCG == 3) rs_level<NVP / 4, 4>(x, lane);
+}
+
+}  // namespace
+
+template <int BITS, int D, int QG>
+__global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __grid_constant__ AttnArgs a) {
+  using C = Dec<BITS, D, QG>;
+  constexpr int CPW = C::CPW, NCG = C::NCG, RPW = C::RPW, TPS = C::TPS, CPL = C::CPL;
+  constexpr int NV = C::NV, NVP = C::NVP, VPL = C::VPL;
+  __shared__ int sm_bs[VARQ_MAX_BLOCKS + 1];
+  __shared__ float sm_q[QG][D];
+  __shared__ float sm_p[kDecWarps][QG][TPS];     // this step's P, read back by every lane
+  __shared__ float sm_o[kDecWarps][QG][D];       // per-warp O for the merge
+  __shared__ float sm_ml[kDecWarps][QG][2];      // per-warp (m, l)
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nrg = (a.lq + QG - 1) / QG;
+  const int rg = blockIdx.x % nrg, split = blockIdx.x / nrg;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = int64_t(b) * a.heads + h;
+  const float sl2 = a.scale_log2;
+
+  for (int i = tid; i <= a.n_cached_blocks; i += kDecThreads) sm_bs[i] = a.block_start[i];
+  for (int i = tid; i < QG * D; i += kDecThreads) {
+    const int g = i / D, d = i % D, row = rg * QG + g;
+    sm_q[g][d] = row < a.lq ? __bfloat162float(a.q[int64_t(b) * a.q_sb + int64_t(h) * a.q_sh + int64_t(row) * a.q_st + d])
+                            : 0.0f;
+  }
+  __syncthreads();
+
+  // this CTA's word rows [w_begin, w_end): ranges of whole warp steps
+  const int t_att = a.t_att;
+  const int words_att = (t_att + CPW - 1) / CPW;
+  const int per = ((words_att + a.n_splits - 1) / a.n_splits + RPW - 1) / RPW * RPW;
+  const int w_begin = min(words_att, split * per), w_end = min(words_att, w_begin + per);
+  const int nsteps = (w_end - w_begin + RPW - 1) / RPW;
+
+  const int r = lane / NCG, cg = lane % NCG;  // K: word row of the step, 16-channel group
+  const uint32_t* kw_base = a.k_packed + bh * a.words_per_row * D;
+  const uint32_t* vw_base = a.v_packed + bh * a.words_per_row * D;
+  const uint32_t* km_base = a.k_meta + bh * a.n_blocks_total * D;
+  const uint32_t* vm_base = a.v_meta + bh * a.n_blocks_total * D;
+
+  // the query, pre-scaled by scale log2 e, for this lane's 16 K channels
+  float qs[QG][16];
+#pragma unroll
+  for (int g = 0; g < QG; ++g)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) qs[g][c] = sm_q[g][cg * 16 + c] * sl2;
+  // (scale, min) of the loaded block: the lane's 16 K channels and its V channels
+  float ks[16], kmn[16], vs[CPL], vmn[CPL];
+  auto set_block = [&](int blk) {
+    const uint4* mk = reinterpret_cast<const uint4*>(km_base + int64_t(blk) * D + cg * 16);
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const uint4 w = __ldg(mk + c4);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 sm = meta_unpack(ws[e]);
+        ks[c4 * 4 + e] = sm.x;
+        kmn[c4 * 4 + e] = sm.y;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const float2 sv = meta_unpack(__ldg(vm_base + int64_t(blk) * D + lane + 32 * k));
+      vs[k] = sv.x;
+      vmn[k] = sv.y;
+    }
+  };
+
+  float m[QG], l[QG], O[QG][CPL];
+#pragma unroll
+  for (int g = 0; g < QG; ++g) {
+    m[g] = -__int_as_float(0x7F800000);
+    l[g] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) O[g][k] = 0.0f;
+  }
+  int cur = -1;  // block whose constants are loaded
+
+  for (int s = warp; s < nsteps; s += kDecWarps) {
+    const int wr0 = w_begin + s * RPW;
+    const int ts = wr0 * CPW;
+    const int te = min(min(wr0 + RPW, w_end) * CPW, t_att);
+    const int wk = wr0 + r;           // this lane's K word row
+    const int tr = wk * CPW;          // its first token
+    // packed words of the step: K row wk, channels cg*16..+15; V rows
+    // wr0..wr0+RPW-1, channels lane + 32 k (rows past the range read as 0)
+    uint32_t kw[16], vw[RPW][CPL];
+    if (wk < w_end) {
+      const uint4* p = reinterpret_cast<const uint4*>(kw_base + int64_t(wk) * D + cg * 16);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint4 w = __ldg(p + c4);
+        kw[c4 * 4] = w.x;
+        kw[c4 * 4 + 1] = w.y;
+        kw[c4 * 4 + 2] = w.z;
+        kw[c4 * 4 + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) kw[c] = 0u;
+    }
+    // V words now, ahead of their use, unless the score sums are wide
+    // (2-bit codes: 16 per word), where the registers go to those instead
+    constexpr bool kEarlyV = NVP <= 8;
+    auto load_v = [&]() {
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+          vw[rr][k] = wr0 + rr < w_end ? __ldg(vw_base + int64_t(wr0 + rr) * D + lane + 32 * k) : 0u;
+    };
+    if (kEarlyV) load_v();
+
+    // block of the step's first token (blocks only move forward); a step
+    // inside one block uses that block's constants, a step across blocks
+    // looks up each token's own (scale, min)
+    int blk = max(cur, 0);
+    while (ts >= sm_bs[blk + 1]) ++blk;
+    const bool across = te > sm_bs[blk + 1];
+    if (!across && blk != cur) {
+      set_block(blk);
+      cur = blk;
+    }
+
+    // ---- scores: K_hat = bf16(fmaf(code, s, min)) as the dequantization
+    // defines it, dotted with the lane's 16 query channels, then summed over
+    // the NCG lanes of the word row; token j of the lane's row is tr + j
+    float acc[NVP];
+#pragma unroll
+    for (int i = 0; i < NVP; ++i) acc[i] = 0.0f;
+    if (!across) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          float k0, k1;
+          dequant_pair<BITS>(kw[c], j, j + 1 < CPW, ks[c], kmn[c], k0, k1);
+#pragma unroll
+          for (int g = 0; g < QG; ++g) {
+            acc[g * CPW + j] = __fmaf_rn(qs[g][c], k0, acc[g * CPW + j]);
+            if (j + 1 < CPW) acc[g * CPW + j + 1] = __fmaf_rn(qs[g][c], k1, acc[g * CPW + j + 1]);
+          }
+        }
+      }
+    } else {
+      int tb[CPW];  // block of each token of the lane's row
+      {
+        int bq = blk;
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          while (bq + 1 < a.n_cached_blocks && tr + j >= sm_bs[bq + 1]) ++bq;
+          tb[j] = bq;
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t w = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + cg * 16 + c) : 0u;
+        float qv[QG];
+#pragma unroll
+        for (int g = 0; g < QG; ++g) qv[g] = sm_q[g][cg * 16 + c] * sl2;
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const float2 sm = meta_unpack(__ldg(km_base + int64_t(tb[j]) * D + cg * 16 + c));
+          const float kh = bf16_round(__fmaf_rn(code_f<BITS>(w, j), sm.x, sm.y));
+#pragma unroll
+          for (int g = 0; g < QG; ++g) acc[g * CPW + j] = __fmaf_rn(qv[g], kh, acc[g * CPW + j]);
+        }
+      }
+    }
+    reduce_scatter<NVP, C::LOG_NCG>(acc, lane);
+
+    // ---- online softmax over this step; the lane's VPL scores are partials
+    // idx = VPL bitrev(cg) + i: row idx / CPW, token tr + idx % CPW
+    const int idx0 = VPL * bitrev<C::LOG_NCG>(cg);
+#pragma unroll
+    for (int g = 0; g < QG; ++g) {
+      float mx = -__int_as_float(0x7F800000);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV && idx / CPW == g && tr + idx % CPW < te) mx = fmaxf(mx, acc[i]);
+      }
+      if (__any_sync(0xFFFFFFFFu, mx > m[g] + kDecRescale)) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        const float mn = fmaxf(m[g], mx);
+        const float alpha = ex2_approx(m[g] - mn);
+        l[g] *= alpha;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) O[g][k] *= alpha;
+        m[g] = mn;
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV && idx / CPW == g) {
+          const int j = idx % CPW;
+          const float p = tr + j < te ? ex2_approx(acc[i] - m[g]) : 0.0f;
+          l[g] += p;
+          sm_p[warp][g][r * CPW + j] = p;
+        }
+      }
+    }
+    __syncwarp();
+    if (!kEarlyV) load_v();
+
+    // ---- O += P V_hat with V_hat = bf16(fmaf(code, s, min)); tokens past
+    // the range have P = 0
+    if (!across) {
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+#pragma unroll
+        for (int j = 0; j < CPW; j += 2) {
+          float p0[QG], p1[QG];
+#pragma unroll
+          for (int g = 0; g < QG; ++g) {
+            p0[g] = sm_p[warp][g][rr * CPW + j];
+            p1[g] = j + 1 < CPW ? sm_p[warp][g][rr * CPW + j + 1] : 0.0f;
+          }
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            float v0, v1;
+            dequant_pair<BITS>(vw[rr][k], j, j + 1 < CPW, vs[k], vmn[k], v0, v1);
+#pragma unroll
+            for (int g = 0; g < QG; ++g) {
+              O[g][k] = __fmaf_rn(p0[g], v0, O[g][k]);
+              if (j + 1 < CPW) O[g][k] = __fmaf_rn(p1[g], v1, O[g][k]);
+            }
+          }
+        }
+      }
+    } else {
+      int bq = blk;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const int t = ts + rr * CPW + j;
+          while (bq + 1 < a.n_cached_blocks && t >= sm_bs[bq + 1]) ++bq;
+          float pg[QG];
+#pragma unroll
+          for (int g = 0; g < QG; ++g) pg[g] = sm_p[warp][g][rr * CPW + j];
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const float2 sm = meta_unpack(__ldg(vm_base + int64_t(bq) * D + lane + 32 * k));
+            const float vh = bf16_round(__fmaf_rn(code_f<BITS>(vw[rr][k], j), sm.x, sm.y));
+#pragma unroll
+            for (int g = 0; g < QG; ++g) O[g][k] = __fmaf_rn(pg[g], vh, O[g][k]);
+          }
+        }
+      }
+    }
+    __syncwarp();  // sm_p is rewritten by the next step
+  }
+
+  // ---- merge the warps' (m, l, O) into this range's partial
+#pragma unroll
+  for (int g = 0; g < QG; ++g) {
+    float ls = l[g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o);
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) sm_o[warp][g][lane + 32 * k] = O[g][k];
+    if (lane == 0) {
+      sm_ml[warp][g][0] = m[g];
+      sm_ml[warp][g][1] = ls;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < QG * D; i += kDecThreads) {
+    const int g = i / D, d = i % D, row = rg * QG + g;
+    if (row >= a.lq) continue;
+    float M = -__int_as_float(0x7F800000);
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_ml[w][g][0]);
+    float o = 0.0f, L = 0.0f;
+    if (M != -__int_as_float(0x7F800000)) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mw = sm_ml[w][g][0];
+        if (mw == -__int_as_float(0x7F800000)) continue;
+        const float f = ex2_approx(mw - M);
+        o = __fmaf_rn(f, sm_o[w][g][d], o);
+        L = __fmaf_rn(f, sm_ml[w][g][1], L);
+      }
+    }
+    float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
+                int64_t(row) * (D + 2);
+    ws[d] = o;
+    if (d == 0) {
+      ws[D] = M;
+      ws[D + 1] = L;
+    }
+  }
+}
+
+namespace {
+
+// Query rows per CTA (more rows run as more row groups over the same range).
+constexpr int kDecQG = 1;
+
+template <int BITS, int D, int QG>
+cudaError_t launch_dec(const AttnArgs& a, cudaStream_t stream) {
+  const int nrg = (a.lq + QG - 1) / QG;
+  const dim3 grid(unsigned(nrg * a.n_splits), unsigned(a.heads), unsigned(a.batch));
+  attn_decode_kernel<BITS, D, QG><<<grid, kDecThreads, 0, stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attention_combine(a, stream);
+}
+
+template <int BITS>
+cudaError_t launch_dec_bits(const AttnArgs& a, cudaStream_t s) {
+  if (a.head_dim == 128) return launch_dec<BITS, 128, kDecQG>(a, s);
+  if (a.head_dim == 64) return launch_dec<BITS, 64, kDecQG>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool use_decode_kernel(const AttnArgs& a) {
+  return a.kv_split && a.rope_cos == nullptr && a.lq <= kDecodeMaxLq;
+}
+
+// About six CTAs per SM over the grid, each warp at least four steps long.
+int split_kv_decode_splits(const AttnArgs& a) {
+  const int nrg = (a.lq + kDecQG - 1) / kDecQG;
+  const int cpw = 32 / a.bits;
+  const int rpw = 32 / (a.head_dim / 16);
+  const int words = (a.t_att + cpw - 1) / cpw;
+  const int64_t base = int64_t(nrg) * a.heads * a.batch;
+  int64_t want = (6 * 148 + base - 1) / base;
+  want = std::min<int64_t>(want, std::max(1, words / (kDecWarps * 4 * rpw)));
+  want = std::max<int64_t>(1, std::min<int64_t>(want, 64));
+  const int per = static_cast<int>((words + want - 1) / want);
+  return (words + per - 1) / per;
+}
+
+cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream) {
+  switch (a.bits) {
+    case 2: return launch_dec_bits<2>(a, stream);
+    case 3: return launch_dec_bits<3>(a, stream);
+    case 4: return launch_dec_bits<4>(a, stream);
+    case 5: return launch_dec_bits<5>(a, stream);
+    case 6: return launch_dec_bits<6>(a, stream);
+    case 7: return launch_dec_bits<7>(a, stream);
+    case 8: return launch_dec_bits<8>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace varq

@@ -126,7 +126,15 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.kv_split = 1;
-  a.n_splits = varq::split_kv_splits(a);
+  // the CUDA-core kernel on the packed codes where it applies and its
+  // partials fit the fixed scratch array, else the tensor-core kernel
+  bool dec = varq::use_decode_kernel(a);
+  if (dec) {
+    a.n_splits = varq::split_kv_decode_splits(a);
+    dec = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits) <=
+          VARQ_NOALLOC_SCRATCH_BYTES;
+  }
+  if (!dec) a.n_splits = varq::split_kv_splits(a);
 
   // the shape must fit the fixed scratch array
   const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits);
@@ -135,6 +143,7 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   rc = scratch_on_current_device(&scratch);
   if (rc != VARQ_OK) return rc;
   a.workspace = scratch;
-  const cudaError_t e = varq::launch_attention_tc(a, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = dec ? varq::launch_attention_decode(a, static_cast<cudaStream_t>(stream))
+                            : varq::launch_attention_tc(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VARQ_OK : VARQ_ERR_CUDA;
 }

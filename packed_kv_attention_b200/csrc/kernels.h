@@ -87,5 +87,12 @@ int split_kv_splits(const AttnArgs& a);
 size_t split_kv_workspace_bytes(int batch, int heads, int lq, int head_dim, int n_splits);
 // The log-sum-exp merge of the split-KV partials into out (and lse).
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t stream);
+// Split-KV form on the CUDA cores straight from the packed codes (no
+// dequantized tile), for short query blocks without pre-RoPE keys; writes the
+// same partials and runs the same merge.
+constexpr int kDecodeMaxLq = 2;
+bool use_decode_kernel(const AttnArgs& a);
+int split_kv_decode_splits(const AttnArgs& a);
+cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace varq

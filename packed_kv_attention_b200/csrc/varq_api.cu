@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/varq.h: argument validation,
 // layout planning and kernel dispatch.  No allocation, no global state.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -178,7 +179,10 @@ size_t varq_packed_attention_workspace(const varq_cache_layout* L, int lq, int n
   if (choose_path(lq, path) != VARQ_PATH_SPLIT || lq > VARQ_SPLIT_MAX_LQ) return 0;
   AttnArgs a;
   fill_attn(a, L, lq, n_cached_blocks);
-  return varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, varq::split_kv_splits(a));
+  // enough for either kernel of the split-KV form (the choice also depends on
+  // the rope tables, which this query does not see)
+  const int n = std::max(varq::split_kv_splits(a), varq::split_kv_decode_splits(a));
+  return varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, n);
 }
 
 int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st,
@@ -229,14 +233,16 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p == VARQ_PATH_TENSOR) return launch_status(varq::launch_attention_tc(a, s));
 
-  // split-KV form: the tensor-core kernel over ranges of KV tiles, then the merge
+  // split-KV form: ranges of the cache over CTAs (the CUDA-core kernel on the
+  // packed codes, or the tensor-core kernel with pre-RoPE keys), then the merge
   a.kv_split = 1;
-  a.n_splits = varq::split_kv_splits(a);
+  const bool dec = varq::use_decode_kernel(a);
+  a.n_splits = dec ? varq::split_kv_decode_splits(a) : varq::split_kv_splits(a);
   const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits);
   if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
   a.workspace = static_cast<float*>(workspace);
-  return launch_status(varq::launch_attention_tc(a, s));
+  return launch_status(dec ? varq::launch_attention_decode(a, s) : varq::launch_attention_tc(a, s));
 }
 
 }  // extern "C"

@@ -171,6 +171,64 @@ def test_attention_pre_rope_keys(path, lq, D):
         _check(out, lse, ref, ref_lse, 0, h, rows)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("lq", [1, 2])
+def test_attention_decode_from_codes(bits, D, lq):
+    """Split-KV form for one or two query rows (the CUDA-core kernel on the
+    packed codes): block boundaries inside packed words, blocks shorter than a
+    word, a ragged end, several KV ranges per head."""
+    B, H = 2, 3
+    sizes = [1, 3, 50, 7, 300, 33, 2, 611]
+    bs = synth.block_starts(sizes)
+    k, v, q, _, _ = _inputs(B, H, D, sizes, lq, seed=bits * 10 + D + lq)
+    L = V.varq_cache_alloc(B, H, D, bits, bs)
+    out, lse = _gpu_attention(L, k, v, q, len(sizes), path=V.PATH_SPLIT)
+    rows = np.arange(lq)
+    for b in range(B):
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), b, h, rows)
+            _check(out, lse, ref, ref_lse, b, h, rows)
+
+
+def _spiked_inputs(B, H, D, T, lq, spikes, seed):
+    """Keys and values ~ N(0, 1), queries sharing a direction u; token t of
+    every (b, h) gets key beta * u for each (t, beta) in spikes, so its score
+    sits about 16 * beta (log2 units) above the background."""
+    g = torch.Generator()
+    g.manual_seed(seed)
+    u = torch.randn(D, generator=g)
+    k = torch.randn(B, H, T, D, generator=g)
+    v = torch.randn(B, H, T, D, generator=g)
+    q = u + 0.3 * torch.randn(B, H, lq, D, generator=g)
+    for t, beta in spikes:
+        k[:, :, t] = beta * u
+    return k.to(torch.bfloat16), v.to(torch.bfloat16), q.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("bits", [4, 3, 8])
+@pytest.mark.parametrize("path,lq", [(V.PATH_TENSOR, 256), (V.PATH_SPLIT, 4), (V.PATH_SPLIT, 1)])
+def test_attention_rising_scores(bits, path, lq):
+    """Scores that jump far above the running maximum inside later KV tiles,
+    at the first, an odd and a later 16-column piece, and in the last partial
+    tile: the running-offset form of the softmax and its exact fallback."""
+    D, B, H = 128, 1, 2
+    sizes = [600, 700, 300]
+    T = sum(sizes)
+    unit = math.lcm(32 // bits, 16)  # KV tile: whole words of whole 16-token MMA slices
+    nkv = (128 // unit) * unit
+    spikes = [(2 * nkv + 0 * 16 + 3, 0.6), (4 * nkv + 3 * 16 + 9, 1.0), (7 * nkv + 2 * 16 + 1, 2.5),
+              (9 * nkv + 1 * 16 + 5, 4.0), (T - 7, 6.0)]
+    k, v, q = _spiked_inputs(B, H, D, T, lq, spikes, seed=bits)
+    bs = synth.block_starts(sizes)
+    L = V.varq_cache_alloc(B, H, D, bits, bs)
+    out, lse = _gpu_attention(L, k, v, q, len(sizes), path=path)
+    rows = np.arange(lq)
+    for h in range(H):
+        ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), 0, h, rows)
+        _check(out, lse, ref, ref_lse, 0, h, rows)
+
+
 def test_attention_custom_scale_and_determinism():
     D, bits, sizes, lq = 128, 4, [64, 300], 150
     bs = synth.block_starts(sizes)
