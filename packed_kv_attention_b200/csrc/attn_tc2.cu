@@ -12,9 +12,14 @@
 //     of the tile for every channel (one 64-token panel, row = channel);
 //   V (B of O = P V, N = channels): rank r holds channels [r D/2, (r+1) D/2)
 //     for every token of the tile.
-// Rank 0's MMA warp waits for both halves (rank 1's dequant and softmax
-// threads arrive on rank 0's barriers across the cluster) and commits to the
-// barriers of both CTAs at once.  The producer of each CTA copies only its
+// Rank 0's MMA warp waits for both halves and commits to the barriers of both
+// CTAs at once.  An mbarrier arrive with cluster-scope release costs the
+// arriving thread about a thousand cycles, so no dequant or softmax thread
+// makes one: every thread arrives on its own CTA's barrier, and in rank 1 one
+// relay thread per stream waits there and forwards a single arrive to rank
+// 0's barrier (warp kRelayWarp: K and V tiles, in the order the dequant warps
+// finish them; the MMA warp, idle in rank 1: P of query tile 0, then 1, per
+// KV tile, the order rank 0's MMA warp consumes them).  The producer of each CTA copies only its
 // halves of the packed words: its K word rows whole, and its half of every V
 // word row.
 #include <algorithm>
@@ -81,10 +86,13 @@ struct Cfg2 {
   static_assert(HALF % GT == 0 && NW % 2 == 0, "each CTA's K half is whole groups of whole words");
 };
 
+constexpr int kRelayWarp = 18;
+constexpr int kThreads2 = kThreads + 32;
+
 }  // namespace
 
 template <int BITS, int D, int NQ, bool ROPE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     attn_tc2_kernel(const __grid_constant__ AttnArgs a) {
   using C = Cfg2<BITS, D, NQ>;
   constexpr int CPW = C::CPW;
@@ -121,19 +129,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->empty[i], kDequantThreads);
-      mbar_init(&bars->kready[i], 2 * kDequantThreads);  // both CTAs' halves (rank 0's barrier)
+      // rank 0: its dequant threads + rank 1's relay; rank 1: its dequant threads
+      mbar_init(&bars->kready[i], kDequantThreads + (rank == 0 ? 1 : 0));
       mbar_init(&bars->kfree[i], 1);
-      mbar_init(&bars->vready[i], 2 * kDequantThreads);
+      mbar_init(&bars->vready[i], kDequantThreads + (rank == 0 ? 1 : 0));
       mbar_init(&bars->vfree[i], 1);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_ready[i], 256);                 // both CTAs' rows of tile i
+      mbar_init(&bars->p_ready[i], 128 + (rank == 0 ? 1 : 0));  // this CTA's rows of tile i (+ relay)
       mbar_init(&bars->o_done[i], 1);
     }
     mbar_init(&bars->teardown, 1);
     bars->abort_flag = 0;
     mbar_fence_init();
   }
-  for (int i = tid; i <= a.n_cached_blocks; i += kThreads) sm_bs[i] = a.block_start[i];
+  for (int i = tid; i <= a.n_cached_blocks; i += kThreads2) sm_bs[i] = a.block_start[i];
   if (warp == kMmaWarp) {  // the same warp in both CTAs
     tmem2_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem2_relinquish();
@@ -142,7 +151,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   {
     const __nv_bfloat16* qg = a.q + int64_t(b) * a.q_sb + int64_t(h) * a.q_sh;
     constexpr int CH = D / 8;
-    for (int idx = tid; idx < NQ * BM * CH; idx += kThreads) {
+    for (int idx = tid; idx < NQ * BM * CH; idx += kThreads2) {
       const int r = idx / CH, c = idx % CH;
       const int row = qblk * (NQ * BM) + r;
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -251,8 +260,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mma2_commit_both(&bars->teardown);
       mbar_wait(&bars->teardown, 0, abort_flag);
     } else if (lane == 0) {
-      // rank 1: its TMEM is released only once the pair's MMAs have finished
+      // rank 1: relay P(j) of each query tile to rank 0, then keep TMEM until
+      // the pair's MMAs have finished
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j)
+        for (int i = 0; i < NQ && ok; ++i) {
+          ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
+          if (ok) mbar_arrive_rank(&bars->p_ready[i], 0);
+        }
       mbar_wait(&bars->teardown, 0, abort_flag);
+    }
+  } else if (warp == kRelayWarp) {
+    // ------------------------------------------------------------- relay
+    if (rank == 1 && lane == 0) {
+      for (int j = 0; j < ntiles; ++j) {
+        if (!mbar_wait(&bars->kready[j % C::KST], (j / C::KST) & 1, abort_flag)) break;
+        mbar_arrive_rank(&bars->kready[j % C::KST], 0);
+        if (!mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag)) break;
+        mbar_arrive_rank(&bars->vready[j % C::VST], 0);
+      }
     }
   } else if (warp >= kDequantWarp0) {
     // ------------------------------------------------------------- dequant
@@ -388,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         fence_async_smem();
-        mbar_arrive_rank(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf], 0);
+        mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
       }
       if (!ok || *abort_flag) break;
       mbar_arrive(&bars->empty[st]);
@@ -513,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive_rank(&bars->p_ready[i], 0);
+      mbar_arrive(&bars->p_ready[i]);
       {
         float r0, r1;
         f2_unpack(rs2, r0, r1);
@@ -598,7 +624,7 @@ cudaError_t launch_tc2(const AttnArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int pairs = (a.lq + 2 * NQ * BM - 1) / (2 * NQ * BM) * (a.kv_split ? a.n_splits : 1);
   dim3 grid(unsigned(2 * pairs), a.heads, a.batch);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(a);
+  kern<<<grid, kThreads2, C::SMEM, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || !a.kv_split) return e;
   return launch_attention_combine(a, stream);
