@@ -54,15 +54,35 @@ __device__ __forceinline__ float code_f(uint32_t w, int j) {
   return small_uint_to_float((w >> (j * BITS)) & ((1u << BITS) - 1u));
 }
 
+// The same without a shift per code: a code at bit offset o (o + BITS <= 23)
+// is OR-ed in place into the mantissa of 2^23, giving 2^23 + c 2^o, and
+// fma(that, 2^-o, -2^(23-o)) = c exactly (a power-of-two scaling and an exact
+// difference); codes above bit 23 come from the word shifted right once by
+// kHighShift<BITS>.  One logic op per code (plus one shift per word) instead
+// of two, the rest on the FMA pipe.
+template <int BITS>
+constexpr int kHighShift = ((23 - BITS) / BITS + 1) * BITS;  // offset of the first code past bit 23
+
+template <int BITS>
+__device__ __forceinline__ float code_in_place(uint32_t w, uint32_t w_hi, int j) {
+  const int o = j * BITS;
+  const bool hi = o + BITS > 23;
+  const int oo = hi ? o - kHighShift<BITS> : o;
+  const uint32_t f = ((hi ? w_hi : w) & (((1u << BITS) - 1u) << oo)) | 0x4B000000u;
+  return __fmaf_rn(__uint_as_float(f), __uint_as_float(uint32_t(127 - oo) << 23),
+                   -__uint_as_float(uint32_t(127 + 23 - oo) << 23));
+}
+
 // fp32 rounded to the nearest bf16 (ties to even), as fp32.
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 // Codes j and j + 1 of a word dequantized as fmaf(code, s, min) and rounded
 // to bf16 together (the second only when `two`).
 template <int BITS>
-__device__ __forceinline__ void dequant_pair(uint32_t w, int j, bool two, float s, float mn, float& x0, float& x1) {
-  const float a = __fmaf_rn(small_uint_to_float((w >> (j * BITS)) & ((1u << BITS) - 1u)), s, mn);
-  const float b = two ? __fmaf_rn(small_uint_to_float((w >> ((j + 1) * BITS)) & ((1u << BITS) - 1u)), s, mn) : 0.0f;
+__device__ __forceinline__ void dequant_pair(uint32_t w, uint32_t w_hi, int j, bool two, float s, float mn, float& x0,
+                                             float& x1) {
+  const float a = __fmaf_rn(code_in_place<BITS>(w, w_hi, j), s, mn);
+  const float b = two ? __fmaf_rn(code_in_place<BITS>(w, w_hi, j + 1), s, mn) : 0.0f;
   const uint32_t u = pack_bf16x2(a, b);
   x0 = __uint_as_float(u << 16);
   x1 = __uint_as_float(u & 0xFFFF0000u);
@@ -233,10 +253,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __gri
     if (!across) {
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
+        const uint32_t w_hi = kw[c] >> kHighShift<BITS>;
 #pragma unroll
         for (int j = 0; j < CPW; j += 2) {
           float k0, k1;
-          dequant_pair<BITS>(kw[c], j, j + 1 < CPW, ks[c], kmn[c], k0, k1);
+          dequant_pair<BITS>(kw[c], w_hi, j, j + 1 < CPW, ks[c], kmn[c], k0, k1);
 #pragma unroll
           for (int g = 0; g < QG; ++g) {
             acc[g * CPW + j] = __fmaf_rn(qs[g][c], k0, acc[g * CPW + j]);
@@ -322,7 +343,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __gri
 #pragma unroll
           for (int k = 0; k < CPL; ++k) {
             float v0, v1;
-            dequant_pair<BITS>(vw[rr][k], j, j + 1 < CPW, vs[k], vmn[k], v0, v1);
+            dequant_pair<BITS>(vw[rr][k], vw[rr][k] >> kHighShift<BITS>, j, j + 1 < CPW, vs[k], vmn[k], v0, v1);
 #pragma unroll
             for (int g = 0; g < QG; ++g) {
               O[g][k] = __fmaf_rn(p0[g], v0, O[g][k]);
