@@ -13,7 +13,8 @@
 //               (= TMEM lane); online softmax in the log2 domain; P is written
 //               back into TMEM over the consumed S columns (16-bit pairs) and
 //               O is rescaled in TMEM only when the row max grows by > 2^8.
-//   warps 8-15  dequant: (channel, part of the tile) per thread; packed words
+//   warps 8-15  dequant (and warps 4-7 when NQ = 1, where no second softmax
+//               warpgroup needs them): (channel, part of the tile) per thread; packed words
 //               + per-block (scale, min) -> exact bf16 values written straight
 //               into the 128-byte swizzled operand layout the MMA reads
 //               (optionally rotating key pairs for the pre-RoPE key mode).
@@ -27,6 +28,10 @@
 //               warpgroup works while the tensor core runs the other tile.
 //               QK_i(j+1) overwrites the TMEM columns PV_i(j) reads P from;
 //               the MMAs of one issuing thread execute in order.
+// With one query tile (NQ = 1) S is double-buffered in TMEM (columns 0 and
+// 128, O at 256): the order per KV tile j is PV(j), QK(j+2) into the buffer
+// P(j) came from, so S(j+1) is ready while the softmax works on tile j and
+// the chain softmax -> PV -> QK -> softmax spans two tiles.
 //
 // Shared-memory operand layouts (16-bit, 128-byte swizzle, 64 elements/row):
 //   Q_i [D/64 panels][128 rows][64]  K-major A of S_i = Q_i K^T
@@ -60,7 +65,10 @@ struct Cfg {
   static constexpr int NW = NKV / CPW;                // packed words per tile
   static constexpr int NG = NKV / GT;                 // dequant groups per tile
   static constexpr int PANELS = (NKV + 63) / 64;
-  static constexpr int TPC = kDequantThreads / D;     // dequant threads per channel
+  // dequant threads: warps 8-15, plus warps 4-7 when there is one query tile
+  // (no second softmax warpgroup)
+  static constexpr int DEQ = NQ == 1 ? kDequantThreads + 128 : kDequantThreads;
+  static constexpr int TPC = DEQ / D;                 // dequant threads per channel
   // codes of a word are taken CPC at a time from a shifted copy, so their
   // bit offsets inside it stay below 2^14
   static constexpr int CPC = BITS == 2 ? 4 : (BITS == 3 ? 3 : (BITS == 8 ? 1 : 2));
@@ -90,7 +98,8 @@ struct Cfg {
   static constexpr uint32_t OFF_STAGE = OFF_V + VST * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_STAGE + PST * STAGE_BYTES;
   static constexpr uint32_t SMEM = OFF_BAR + kBarBytes + 1024;
-  static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
+  static constexpr bool DB = NQ == 1;                 // S double-buffered
+  static constexpr uint32_t TMEM_COLS = 512;
   static_assert(NKV % 16 == 0 && NKV <= 128, "tile shape");
 };
 
@@ -130,10 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->full[i], 1);
-      mbar_init(&bars->empty[i], kDequantThreads);
-      mbar_init(&bars->kready[i], kDequantThreads);
+      mbar_init(&bars->empty[i], C::DEQ);
+      mbar_init(&bars->kready[i], C::DEQ);
       mbar_init(&bars->kfree[i], 1);
-      mbar_init(&bars->vready[i], kDequantThreads);
+      mbar_init(&bars->vready[i], C::DEQ);
       mbar_init(&bars->vfree[i], 1);
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_ready[i], 128);
@@ -166,6 +175,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // TMEM columns: S of query tile i (double-buffered: buffer j & 1 of KV
+  // tile j at 0 or 128) and O_i
+  auto s_col = [](int i, int j) -> uint32_t { return C::DB ? uint32_t(j & 1) * 128u : col_s(i); };
+  auto o_col = [](int i) -> uint32_t { return C::DB ? 256u : col_o<NQ>(i); };
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = qd + uint64_t(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
           const uint64_t bd = kd + uint64_t((kk * 2048) >> 4);
-          mma_ss(tmem + col_s(i), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + s_col(i, j), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int j) {
@@ -218,36 +231,68 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
         for (int kk = 0; kk < C::NKV / 16; ++kk) {
           const uint64_t bd = vd + uint64_t(((kk >> 2) * (D * 128) + (kk & 3) * 32) >> 4);
-          mma_ts(tmem + col_o<NQ>(i), tmem + col_s(i) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + o_col(i), tmem + s_col(i, j) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        for (int i = 0; i < NQ; ++i) {
-          issue_qk(i, 0);
-          mma_commit(&bars->s_full[i]);
-        }
-        mma_commit(&bars->kfree[0]);
-      }
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag);
-        for (int i = 0; i < NQ && ok; ++i) {
-          ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
+      if constexpr (C::DB) {
+        // one query tile: S(0), S(1) first, then per KV tile j PV(j) and S(j + 2)
+        // into the buffer P(j) is read from (the MMAs run in issue order);
+        // barriers indexed by j & 1
+        bool ok = true;
+        for (int j = 0; j < min(2, ntiles) && ok; ++j) {
+          ok = mbar_wait(&bars->kready[j % C::KST], (j / C::KST) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(i, j);
-          mma_commit(&bars->o_done[i]);
-          if (i == NQ - 1) mma_commit(&bars->vfree[j % C::VST]);
-          if (j + 1 < ntiles) {
-            if (i == 0) {
-              ok = mbar_wait(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_qk(i, j + 1);
+          issue_qk(0, j);
+          mma_commit(&bars->s_full[j & 1]);
+          mma_commit(&bars->kfree[j % C::KST]);
+        }
+        for (int j = 0; j < ntiles && ok; ++j) {
+          ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag) &&
+               mbar_wait(&bars->p_ready[j & 1], (j >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, j);
+          mma_commit(&bars->o_done[j & 1]);
+          mma_commit(&bars->vfree[j % C::VST]);
+          if (j + 2 < ntiles) {
+            ok = mbar_wait(&bars->kready[(j + 2) % C::KST], ((j + 2) / C::KST) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(0, j + 2);
+            mma_commit(&bars->s_full[j & 1]);
+            mma_commit(&bars->kfree[(j + 2) % C::KST]);
+          }
+        }
+      } else {
+        bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < NQ; ++i) {
+            issue_qk(i, 0);
             mma_commit(&bars->s_full[i]);
-            if (i == NQ - 1) mma_commit(&bars->kfree[(j + 1) % C::KST]);
+          }
+          mma_commit(&bars->kfree[0]);
+        }
+        for (int j = 0; j < ntiles && ok; ++j) {
+          ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag);
+          for (int i = 0; i < NQ && ok; ++i) {
+            ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(i, j);
+            mma_commit(&bars->o_done[i]);
+            if (i == NQ - 1) mma_commit(&bars->vfree[j % C::VST]);
+            if (j + 1 < ntiles) {
+              if (i == 0) {
+                ok = mbar_wait(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_qk(i, j + 1);
+              mma_commit(&bars->s_full[i]);
+              if (i == NQ - 1) mma_commit(&bars->kfree[(j + 1) % C::KST]);
+            }
           }
         }
       }
@@ -255,9 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mma_commit(&bars->teardown);
       mbar_wait(&bars->teardown, 0, abort_flag);
     }
-  } else if (warp >= kDequantWarp0) {
+  } else if (warp >= kDequantWarp0 || (NQ == 1 && warp >= 4)) {
     // ------------------------------------------------------------- dequant
-    const int dt = tid - kDequantWarp0 * 32;
+    const int dt = warp >= kDequantWarp0 ? tid - kDequantWarp0 * 32 : kDequantThreads + tid - 128;
     const int d = dt % D;
     const int part = dt / D;
     const int64_t bh = int64_t(b) * a.heads + h;
@@ -389,14 +434,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int i = warp >> 2;                 // query tile of this warpgroup
     const int r = (warp & 3) * 32 + lane;    // row within the tile == TMEM lane
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
-    const uint32_t s_tmem = lane_base + col_s(i);
-    const uint32_t o_tmem = lane_base + col_o<NQ>(i);
+    const uint32_t o_tmem = lane_base + o_col(i);
     const float sl2 = a.scale_log2;
     float m_run = -__int_as_float(0x7F800000);
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      ok = wait_all(&bars->s_full[i], j & 1, abort_flag);
+      // S of this tile: TMEM columns and barrier (buffer j & 1 when double-buffered)
+      const uint32_t s_tmem = lane_base + s_col(i, j);
+      ok = C::DB ? wait_all(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag)
+                 : wait_all(&bars->s_full[i], j & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const int valid = min(C::NKV, t_att - (tile0 + j) * C::NKV);
@@ -434,9 +481,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       float m_new = m_run;
       if (j == 0 || mx > m_run + kRescaleThreshold) m_new = fmaxf(mx, m_run);
       const float alpha = (j == 0) ? 0.0f : ex2_approx(m_run - m_new);
-      // PV_i of the previous tile has finished before O_i is rescaled
-      if (j >= 1) {
-        ok = wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
+      // PV_i of the previous tile has finished before O_i is rescaled.  With S
+      // double-buffered, o_done[t & 1] completes once per PV(t) of that
+      // parity; a wait names tile t's phase, exact while tile t - 2's has been
+      // waited for and PV(t + 2) cannot have run: PV(j - 2) is waited for every
+      // tile (long finished), PV(j - 1) only to rescale O.
+      if (C::DB && j >= 2) {
+        ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag);
+        if (!ok) break;
+      }
+      if (j >= 1 && (!C::DB || __any_sync(0xFFFFFFFFu, m_new != m_run))) {
+        ok = C::DB ? wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)
+                   : wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xFFFFFFFFu, m_new != m_run)) {
@@ -504,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready[i]);
+      mbar_arrive(C::DB ? &bars->p_ready[j & 1] : &bars->p_ready[i]);
       {
         float r0, r1;
         f2_unpack(rs2, r0, r1);
@@ -514,13 +570,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       m_run = m_new;
     }
     // ------------------------------------------------------------- epilogue
+    // O_i is final once the last PV_i has completed (double-buffered S: PV of
+    // the last two tiles, waited for in order)
+    auto o_final = [&]() {
+      if constexpr (C::DB) {
+        return (ntiles < 2 || wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, abort_flag)) &&
+               wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag);
+      } else {
+        return wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
+      }
+    };
     if (a.kv_split) {
       // split-KV form: the unnormalised partial of this KV range (O, running
       // max m in the log2 domain, running sum l); m = -inf marks "no token"
       const int row = qblk * (NQ * BM) + i * BM + r;
       float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
                   int64_t(row) * (D + 2);
-      const bool have = ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
+      const bool have = ok && ntiles > 0 && o_final();
       if (have) {
         tc_fence_after();
 #pragma unroll 1
@@ -540,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         ws[D] = have ? m_run : -__int_as_float(0x7F800000);
         ws[D + 1] = have ? l_run : 0.0f;
       }
-    } else if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag)) {
+    } else if (ok && ntiles > 0 && o_final()) {
       tc_fence_after();
       const int row = qblk * (NQ * BM) + i * BM + r;
       const float inv = 1.0f / l_run;
@@ -584,10 +650,13 @@ template <int BITS, int D, int NQ, bool ROPE>
 cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<BITS, D, NQ>;
   auto kern = attn_tc_kernel<BITS, D, NQ, ROPE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  // every CTA allocates all 512 TMEM columns: ask for enough shared memory
+  // that no second CTA is placed on the SM to wait for them
+  const uint32_t smem = std::max<uint32_t>(C::SMEM, kSmemUsable / 2 + 1024);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned((a.lq + NQ * BM - 1) / (NQ * BM) * (a.kv_split ? a.n_splits : 1)), a.heads, a.batch);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(a);
+  kern<<<grid, kThreads, smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || !a.kv_split) return e;
   return launch_attention_combine(a, stream);

@@ -29,13 +29,15 @@ struct Barriers {
   uint64_t full[2], empty[2];     // packed stage filled by TMA / released by dequant
   uint64_t kready[2], kfree[2];   // 16-bit K tile written / consumed by all S MMAs
   uint64_t vready[2], vfree[2];   // 16-bit V tile written / consumed by all PV MMAs
-  uint64_t s_full[2];             // S_i of the current tile in TMEM
+  // indexed by query tile i, or by KV tile & 1 where S is double-buffered
+  uint64_t s_full[2];             // S_i of a KV tile in TMEM
   uint64_t p_ready[2];            // P_i in TMEM and O_i rescaled
   uint64_t o_done[2];             // PV_i finished
   uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(Barriers) <= 512, "the barriers sit below the block-start table");
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const bool ok = mbar_wait(bar, parity, abort_flag);
