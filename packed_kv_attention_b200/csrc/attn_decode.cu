@@ -445,17 +445,33 @@ bool use_decode_kernel(const AttnArgs& a) {
   return a.kv_split && a.rope_cos == nullptr && a.lq <= kDecodeMaxLq;
 }
 
-// About six CTAs per SM over the grid, each warp at least four steps long.
+// About six CTAs per SM over the grid, each warp at least four steps long;
+// then, up to twice that many ranges, the count that fills the last wave of
+// 148 SMs x 2 resident CTAs (128 registers a thread) best.
 int split_kv_decode_splits(const AttnArgs& a) {
   const int nrg = (a.lq + kDecQG - 1) / kDecQG;
   const int cpw = 32 / a.bits;
   const int rpw = 32 / (a.head_dim / 16);
   const int words = (a.t_att + cpw - 1) / cpw;
   const int64_t base = int64_t(nrg) * a.heads * a.batch;
+  const int64_t cap_len = std::max(1, words / (kDecWarps * 4 * rpw));
   int64_t want = (6 * 148 + base - 1) / base;
-  want = std::min<int64_t>(want, std::max(1, words / (kDecWarps * 4 * rpw)));
+  want = std::min<int64_t>(want, cap_len);
   want = std::max<int64_t>(1, std::min<int64_t>(want, 64));
-  const int per = static_cast<int>((words + want - 1) / want);
+  const int64_t cap = std::min<int64_t>(std::min<int64_t>(2 * want, 64), cap_len);
+  constexpr int64_t kSlots = 148 * 2;
+  int best = static_cast<int>(want);
+  double best_eff = 0.0;
+  for (int64_t s = want; s <= std::max(want, cap); ++s) {
+    const int per_s = static_cast<int>((words + s - 1) / s);
+    const int64_t n = ((words + per_s - 1) / per_s) * base;
+    const double eff = double(n) / double(kSlots * ((n + kSlots - 1) / kSlots));
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = static_cast<int>(s);
+    }
+  }
+  const int per = (words + best - 1) / best;
   return (words + per - 1) / per;
 }
 

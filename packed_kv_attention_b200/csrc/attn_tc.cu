@@ -706,7 +706,8 @@ bool use_pair_kernel(const AttnArgs& a) { return a.rope_cos != nullptr && !a.kv_
 
 // Split-KV form: enough CTAs for about two waves over 148 SMs (one CTA per
 // SM), each range at least four KV tiles long when the cache allows, and no
-// empty range.
+// empty range; then, up to twice that many ranges, the count that fills the
+// last wave best.
 int split_kv_splits(const AttnArgs& a) {
   const int nkv = tile_tokens(a.bits);
   const int ntiles = (a.t_att + nkv - 1) / nkv;
@@ -715,7 +716,20 @@ int split_kv_splits(const AttnArgs& a) {
   want = std::min<int64_t>(want, std::max(1, ntiles / 4));
   want = std::min<int64_t>(want, 64);
   want = std::max<int64_t>(want, 1);
-  const int per = static_cast<int>((ntiles + want - 1) / want);
+  // among want .. 2 want ranges, the count whose last wave over 148 SMs is fullest
+  const int64_t cap = std::min<int64_t>(std::min<int64_t>(2 * want, 64), std::max(1, ntiles / 4));
+  int best = static_cast<int>(want);
+  double best_eff = 0.0;
+  for (int64_t s = want; s <= std::max(want, cap); ++s) {
+    const int per_s = static_cast<int>((ntiles + s - 1) / s);
+    const int64_t n = ((ntiles + per_s - 1) / per_s) * base;
+    const double eff = double(n) / double(148 * ((n + 147) / 148));
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = static_cast<int>(s);
+    }
+  }
+  const int per = (ntiles + best - 1) / best;
   return (ntiles + per - 1) / per;
 }
 
