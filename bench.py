@@ -407,13 +407,102 @@ def measure_rows(dev, stream, peaks, iters=5):
         attn()
     t = statistics.median(_event_times(attn, stream, 3))
     fl = attention_flops(w, w.lq[-1])
+
+    # the same layer with keys rotated before quantization (post-RoPE cache):
+    # no tables, the plain tensor path; the cost comparison of the two modes
+    def attn_post():
+        V.varq_packed_attention(pipe.L, pipe.q, pipe.kp, pipe.km, pipe.vp, pipe.vm, pipe.out,
+                                workspace=pipe.ws, dev_status=st, stream=stream)
+    for _ in range(2):
+        attn_post()
+    t_post = statistics.median(_event_times(attn_post, stream, 3))
     rows["a8_pre_rope_attention"] = {
         "workload": f"self_forcing: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} Lq={w.lq[-1]} INT4 pre-RoPE",
         "bound": "tensor", "ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12,
-        "frac_tensor": fl / (t * 1e-3) / 1e12 / tflops_peak}
-    rows["device_status"] = int(st.item())
+        "frac_tensor": fl / (t * 1e-3) / 1e12 / tflops_peak,
+        "post_rope_ms": t_post, "post_rope_TFLOP/s": fl / (t_post * 1e-3) / 1e12}
     del pipe
     torch.cuda.empty_cache()
+
+    # generation loop (a step beyond the path's single call): per generation
+    # block, quantize+pack its K and V into the preallocated caches, then its
+    # queries attend to all blocks so far; whole loop timed, INT4
+    from packed_kv_attention_b200.generation import PackedKVLoop
+    loops = {}
+    for name in ("var_d16", "infinity_8b"):
+        w = synth.WORKLOADS[name]
+        data = synth.make_inputs(w, lq=1, seed=5, device=dev)
+        k, v, bs = data["k"], data["v"], data["block_start"]
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        qs = [torch.randn(w.batch, w.heads, n, w.head_dim, generator=g, device=dev).to(torch.bfloat16)
+              for n in w.block_sizes]
+        outs = [torch.empty_like(q) for q in qs]
+        loop = PackedKVLoop(w.batch, w.heads, w.head_dim, 4, w.block_sizes, device=dev)
+        torch.cuda.synchronize()  # inputs and buffers were made on the default stream
+
+        def run_loop():
+            for i in range(len(w.block_sizes)):
+                loop.step(i, k[:, :, bs[i]:bs[i + 1]], v[:, :, bs[i]:bs[i + 1]], qs[i], out=outs[i], stream=stream)
+        run_loop()
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2, written between timed loops
+        times = []
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run_loop()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        t = statistics.median(times)
+        # the same loop captured once in a CUDA graph and replayed (launch costs
+        # leave the host); the library makes no allocation or synchronisation
+        graph_ms, graph_note = None, None
+        try:
+            ref = [o.clone() for o in outs]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                run_loop()
+            with torch.cuda.stream(stream):  # replay() runs on the current stream
+                for o in outs:
+                    o.zero_()
+                graph.replay()
+            torch.cuda.synchronize()
+            if not all(torch.equal(o, r) for o, r in zip(outs, ref)):
+                raise RuntimeError("graph replay did not reproduce the loop's outputs")
+            gtimes = []
+            for _ in range(3):
+                with torch.cuda.stream(stream):
+                    flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                with torch.cuda.stream(stream):
+                    graph.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                gtimes.append(a.elapsed_time(b))
+            graph_ms = statistics.median(gtimes)
+            del graph, ref
+        except Exception as e:  # capture not possible here: keep the stream-launched time only
+            graph_note = f"{type(e).__name__}: {str(e)[:160]}"
+            torch.cuda.synchronize()
+        del flush
+        fl = sum(4.0 * w.batch * w.heads * n * bs[i + 1] * w.head_dim for i, n in enumerate(w.block_sizes))
+        loops[name] = {"steps": len(w.block_sizes), "ms": t, "ms_per_step": t / len(w.block_sizes),
+                       "attention_TFLOP": fl / 1e12, "TFLOP/s": fl / (t * 1e-3) / 1e12,
+                       "graph_ms": graph_ms, "device_status": loop.device_status()}
+        if graph_note:
+            loops[name]["graph_note"] = graph_note
+        del data, k, v, qs, outs, loop
+        torch.cuda.empty_cache()
+    rows["next_generation_loop"] = {
+        "workload": "VAR-d16-like (B1 H16 D64, 10 blocks, T=680) and Infinity-8B-like (B2 H32 D128, 13 blocks, "
+                    "T=10521); each step: quantize+pack K, V of block k, then its queries over blocks 0..k; INT4; "
+                    "L2 flushed before each timed loop",
+        **loops}
+    rows["device_status"] = int(st.item())
     return rows
 
 

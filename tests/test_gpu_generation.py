@@ -1,0 +1,77 @@
+"""The generation loop over the packed KV cache (packed_kv_attention_b200.generation):
+one block's keys and values appended per step, then the block's queries attend to
+every cached block — each step against the fp64 oracle over the same prefix."""
+import numpy as np
+import pytest
+import torch
+
+from packed_kv_attention_b200 import synth
+from packed_kv_attention_b200.generation import PackedKVLoop
+from test_gpu_attention import DEV, _check, _oracle_attention
+
+pytestmark = pytest.mark.gpu
+
+
+def _cache(seed, B, H, sizes, D):
+    g = torch.Generator()
+    g.manual_seed(seed)
+    k = synth.kv_cache(g, B, H, sizes, D, 4, 10.0, 50.0)
+    v = synth.kv_cache(g, B, H, sizes, D, 4, 10.0, 50.0)
+    return g, k, v
+
+
+# VAR-like schedule (query blocks of 1, 4 and 9 rows take the split-KV kernels,
+# the rest the tensor-core path), an Infinity-like prefix, block lengths that
+# are not whole words
+@pytest.mark.parametrize("bits,D,sizes", [(4, 64, [1, 4, 9, 16, 25, 36, 64, 100, 169, 256]),
+                                          (2, 128, [1, 4, 16, 36, 64, 144, 256]),
+                                          (3, 128, [5, 150, 7, 300])])
+def test_generation_loop(bits, D, sizes):
+    B, H = 1, 4
+    g, k, v = _cache(bits * 100 + D, B, H, sizes, D)
+    bs = synth.block_starts(sizes)
+    loop = PackedKVLoop(B, H, D, bits, sizes, device=DEV)
+    kd, vd = k.to(DEV), v.to(DEV)
+    for step, n in enumerate(sizes):
+        q = synth.queries(g, B, H, n, D)
+        lse = torch.empty(B, H, n, dtype=torch.float32, device=DEV)
+        out = loop.step(step, kd[:, :, bs[step]:bs[step + 1]], vd[:, :, bs[step]:bs[step + 1]], q.to(DEV), lse=lse)
+        torch.cuda.synchronize()
+        rows = np.arange(n)
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k, v, q, bs, bits, step + 1, 0, h, rows)
+            _check(out, lse, ref, ref_lse, 0, h, rows)
+    assert loop.device_status() == 0
+
+
+def test_generation_loop_chunk_overwrite():
+    """A cached block quantized again from new values (chunk overwrite): later
+    attention sees the new block and its neighbours' shared words intact."""
+    bits, D, B, H = 4, 128, 2, 2
+    sizes = [64, 97, 130, 203]
+    g, k, v = _cache(7, B, H, sizes, D)
+    bs = synth.block_starts(sizes)
+    loop = PackedKVLoop(B, H, D, bits, sizes, device=DEV)
+    for step in range(len(sizes)):
+        loop.append(step, k[:, :, bs[step]:bs[step + 1]].to(DEV), v[:, :, bs[step]:bs[step + 1]].to(DEV))
+    _, k_new, v_new = _cache(8, B, H, sizes, D)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, bs[1]:bs[2]] = k_new[:, :, bs[1]:bs[2]]
+    v2[:, :, bs[1]:bs[2]] = v_new[:, :, bs[1]:bs[2]]
+    loop.append(1, k2[:, :, bs[1]:bs[2]].to(DEV), v2[:, :, bs[1]:bs[2]].to(DEV))
+    q = synth.queries(g, B, H, sizes[-1], D)
+    lse = torch.empty(B, H, sizes[-1], dtype=torch.float32, device=DEV)
+    out = loop.attend(q.to(DEV), len(sizes), lse=lse)
+    torch.cuda.synchronize()
+    rows = np.arange(sizes[-1])
+    for b in range(B):
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k2, v2, q, bs, bits, len(sizes), b, h, rows)
+            _check(out, lse, ref, ref_lse, b, h, rows)
+    assert loop.device_status() == 0
+
+
+def test_generation_loop_rejects_uncached_prefix():
+    loop = PackedKVLoop(1, 1, 64, 4, [8, 8], device=DEV)
+    with pytest.raises(RuntimeError):
+        loop.attend(torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16, device=DEV), 1)
