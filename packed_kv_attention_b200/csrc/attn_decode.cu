@@ -1,24 +1,29 @@
 // Split-KV form for short query blocks on the CUDA cores: attention straight
-// from the packed codes (README, "Fused-kernel overhead reduction": attention
-// reads the packed cache itself; project page, "Next-block prediction": every
-// query attends to the whole cache).
+// from the packed words (README, "Fused-kernel overhead reduction": attention
+// reads the packed cache itself; project page, "Quantization, bit packing, and
+// retrieval": values dequantized to BF16; "Next-block prediction": every query
+// attends to the whole cache).
 //
-// With the per-(channel, block) affine code k = s c + m, a score is
-//   q . k_t = sum_d (q_d s_d,b) c_t,d + sum_d q_d m_d,b,
-// so per block the query is scaled once (q~_d = q_d s_d,b scale log2 e) and
-// the second sum is one bias per (block, query row); and the output is
-//   O_d = sum_b [ s_d,b sum_{t in b} p_t c_t,d + m_d,b sum_{t in b} p_t ].
-// No value is dequantized: every code costs an extract, a convert and one
-// FMA per query row, so the kernel streams the packed words at a rate set by
-// those instructions rather than by a 16-bit tile written to shared memory.
+// With one or two query rows the tensor-core kernel pads each MMA from 1 row
+// to 128 and is bound by writing a 16-bit tile to shared memory.  Here every
+// code is dequantized in registers to the value the definition gives,
+// bf16(fmaf(code, scale, min)), and used at once: K codes in a dot product
+// with the query (pre-scaled by softmax scale x log2 e), V codes in O += P V.
+// A code costs a logic op (OR-ed in place into the mantissa of 2^23), three
+// FMA-pipe ops (exact convert, dequant fma, dot-product fma) and half a bf16
+// pack with its unpack; the ALU pipe is the bound.
 //
-// Work split: CTA (KV range, query-row group, head, batch); its 8 warps take
-// steps of RPW word rows in turn, each warp keeping its own online-softmax
-// state (running max m per row, lane-partial sums l, O for the lane's
-// channels), merged across warps at the end into the split-KV partial
-// (O, m, l) that the log-sum-exp merge (attn_combine.cu) reduces over ranges.
-// Scores are in the log2 domain; the running max moves only when a step's
-// scores exceed it by more than kDecRescale, so P <= 2^kDecRescale.
+// Work split: CTA (KV range, query row, head, batch); its 8 warps take steps
+// of RPW word rows in turn.  K: lane (word row, 16-channel group) forms the
+// partial scores of the row's tokens over its channels, and a reduce-scatter
+// over the row's lanes leaves each lane whole scores.  Each warp keeps its own
+// online-softmax state (running max m, lane-partial sums l, O for the lane's
+// channels lane + 32 k), merged across warps at the end into the split-KV
+// partial (O, m, l) that the log-sum-exp merge (attn_combine.cu) reduces over
+// ranges.  Scores are in the log2 domain; the running max moves only when a
+// step's scores exceed it by more than kDecRescale, so P <= 2^kDecRescale.
+// A step across a generation-block boundary looks up each token's own
+// (scale, min) instead of the block constants held in registers.
 #include <algorithm>
 
 #include "common.cuh"
