@@ -176,7 +176,8 @@ VARQ_API int varq_unpack_dequant(const varq_cache_layout* layout, const uint32_t
 
 /*
  * varq_packed_attention_workspace -- bytes of device workspace
- * varq_packed_attention needs for this shape and path (0 if none).
+ * varq_packed_attention needs for this shape and path (0 if none; for the
+ * split path enough for either of its kernels, with or without rope tables).
  */
 VARQ_API size_t varq_packed_attention_workspace(const varq_cache_layout* layout, int lq,
                                        int n_cached_blocks, int path);
@@ -201,7 +202,12 @@ VARQ_API size_t varq_packed_attention_workspace(const varq_cache_layout* layout,
  *                scores) or NULL.
  *   workspace    device memory of varq_packed_attention_workspace() bytes
  *                (may be NULL when that is 0).
- *   path         VARQ_PATH_AUTO, VARQ_PATH_TENSOR or VARQ_PATH_SPLIT.
+ *   path         VARQ_PATH_AUTO (SPLIT for lq <= VARQ_SPLIT_MAX_LQ, else
+ *                TENSOR), VARQ_PATH_TENSOR or VARQ_PATH_SPLIT.  SPLIT divides
+ *                the cache axis over CTAs and merges their partials; with
+ *                lq <= 2 and no rope tables it runs on the CUDA cores straight
+ *                from the packed words, otherwise on the tensor cores.
+ *                Results agree within the attention tolerance either way.
  *   dev_status   device uint32 or NULL (VARQ_DEV_TIMEOUT).
  */
 VARQ_API int varq_packed_attention(const varq_cache_layout* layout,
