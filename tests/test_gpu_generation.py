@@ -75,3 +75,38 @@ def test_generation_loop_rejects_uncached_prefix():
     loop = PackedKVLoop(1, 1, 64, 4, [8, 8], device=DEV)
     with pytest.raises(RuntimeError):
         loop.attend(torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16, device=DEV), 1)
+
+
+def test_generation_loop_captures_in_a_cuda_graph():
+    """The library allocates and synchronises nothing inside its calls, so a
+    whole generation loop captures into one CUDA graph; a replay reproduces the
+    loop's outputs exactly (the kernels are deterministic)."""
+    bits, D, B, H = 4, 64, 1, 4
+    sizes = [1, 4, 9, 16, 25, 36, 64]
+    g, k, v = _cache(21, B, H, sizes, D)
+    bs = synth.block_starts(sizes)
+    kd, vd = k.to(DEV), v.to(DEV)
+    qs = [synth.queries(g, B, H, n, D).to(DEV) for n in sizes]
+    outs = [torch.empty_like(q) for q in qs]
+    loop = PackedKVLoop(B, H, D, bits, sizes, device=DEV)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def run():
+        for i in range(len(sizes)):
+            loop.step(i, kd[:, :, bs[i]:bs[i + 1]], vd[:, :, bs[i]:bs[i + 1]], qs[i], out=outs[i], stream=stream)
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    with torch.cuda.stream(stream):
+        for o in outs:
+            o.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    for o, e in zip(outs, eager):
+        assert torch.equal(o, e)
+    assert loop.device_status() == 0
