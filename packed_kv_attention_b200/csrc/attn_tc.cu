@@ -12,7 +12,7 @@
 //   warps 0-7   softmax: warpgroup i owns query tile i, one row per thread
 //               (= TMEM lane); online softmax in the log2 domain; P is written
 //               back into TMEM over the consumed S columns (16-bit pairs) and
-//               O is rescaled in TMEM only when the row max grows by > 2^8.
+//               O is rescaled in TMEM only when the row max grows by > 2^16.
 //   warps 8-15  dequant (and warps 4-7 when NQ = 1, where no second softmax
 //               warpgroup needs them): (channel, part of the tile) per thread; packed words
 //               + per-block (scale, min) -> exact bf16 values written straight

@@ -14,7 +14,7 @@ constexpr int kDequantThreads = 256;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int BM = 128;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 16.0f;  // log2 units
 constexpr uint32_t kSmemUsable = 227 * 1024 - 1024;  // minus 1 KB to align the base to 1024
 constexpr uint32_t kBarBytes = 2048;
 
