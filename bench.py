@@ -44,10 +44,11 @@ from packed_kv_attention_b200 import synth  # noqa: E402
 METRIC = "fused packed-KV attention TFLOP/s and quant+pack GB/s at INT4/INT2 (% of roofline)"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dominant kernel, from one ncu capture of this bench's workload (summary and
-# command in profiles/attn_tc_kernel__infinity_8b_int4.md).  Reported as the
-# roofline "traffic" only while the kernel's sources hash to the value they
-# had when the counters were taken; otherwise null.
+# dominant kernel (attn_tc_kernel<4,128,2,false> on the Infinity-8B-like INT4
+# layer), from one ncu capture of this bench run with `--steps 2 --warmup 3
+# --also-bits 0 --no-e2e --no-cpu-baseline --no-rows`, the fourth launch of the
+# kernel.  Reported as the roofline "traffic" only while the kernel's sources
+# hash to the value they had when the counters were taken; otherwise null.
 MEASURED_TRAFFIC = {"workload": "infinity_8b", "bits": 4, "lq": 4096, "rope": False,
                     "bytes": 154.668288e6 + 41.806336e6, "sources_sha256_16": "6718e0f95aad3858"}
 TRAFFIC_SOURCES = ("packed_kv_attention_b200/csrc/attn_tc.cu", "packed_kv_attention_b200/csrc/attn_tc_common.cuh",
@@ -268,7 +269,7 @@ def oracle_sample(w, bits, lq, rows, seed=0):
     rsel = np.arange(min(rows, lq))
     cos = data.get("rope_cos")
     from threadpoolctl import threadpool_limits
-    with threadpool_limits(limits=1):  # one host core: numpy's BLAS would otherwise fan out
+    with threadpool_limits(limits=cpu_cores()):  # numpy's BLAS on every core this process may use
         t0 = time.perf_counter()
         hats = []
         for xb in (kb, vb):
@@ -310,7 +311,7 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args),
-        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -341,7 +342,10 @@ def measure_rows(dev, stream, peaks, iters=5):
             next-frame layer (INT4, 4680 queries over 32,760 tokens)."""
     from packed_kv_attention_b200 import varq as V
     hbm = peaks["hbm_gbs"]
-    tflops_peak = peaks["bf16_tflops_sustained"]
+    # kernels here are timed over regions well under a second at full clocks:
+    # the burst peak applies; the sustained (power-capped) one is reported beside
+    tflops_peak = peaks["bf16_tflops"]
+    tflops_sus = peaks["bf16_tflops_sustained"]
     rows = {}
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     w = synth.WORKLOADS["sweep"]
@@ -420,6 +424,7 @@ def measure_rows(dev, stream, peaks, iters=5):
         "workload": f"self_forcing: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} Lq={w.lq[-1]} INT4 pre-RoPE",
         "bound": "tensor", "ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12,
         "frac_tensor": fl / (t * 1e-3) / 1e12 / tflops_peak,
+        "frac_tensor_sustained": fl / (t * 1e-3) / 1e12 / tflops_sus,
         "post_rope_ms": t_post, "post_rope_TFLOP/s": fl / (t_post * 1e-3) / 1e12}
     del pipe
     torch.cuda.empty_cache()
@@ -572,7 +577,10 @@ def main(argv=None):
     qbytes = quant_bytes(pipe.L, w)
     qp_gbs = qbytes / (qp_avg * 1e-3) / 1e9
     abytes = attention_bytes(pipe.L, w, args.lq, pipe.cos is not None)
-    tensor_peak = peaks["bf16_tflops_sustained"]
+    # the timed region lasts tens of milliseconds at full clocks: the burst bf16
+    # peak is the denominator, the sustained one is reported beside it
+    tensor_peak = peaks["bf16_tflops"]
+    tensor_peak_sus = peaks["bf16_tflops_sustained"]
     hbm_peak = peaks["hbm_gbs"]
     roof_time = max(flops / (tensor_peak * 1e12), abytes / (hbm_peak * 1e9))
     bound = "tensor" if flops / (tensor_peak * 1e12) >= abytes / (hbm_peak * 1e9) else "hbm"
@@ -596,7 +604,8 @@ def main(argv=None):
                      "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
                      "frac": (att_tflops / tensor_peak) if bound == "tensor" else
                      (abytes / (at_avg * 1e-3) / 1e9) / hbm_peak,
-                     "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
+                     "peak_source": f"{peaks['source']} ({'bf16_tflops (burst)' if bound == 'tensor' else 'hbm_gbs'})",
+                     "frac_of_sustained_peak": (att_tflops / tensor_peak_sus) if bound == "tensor" else None,
                      "traffic": measured_traffic(w, args.bits, args.lq, pipe.cos is not None),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "clocks": clocks,
@@ -633,8 +642,11 @@ def main(argv=None):
             dt_tot += dt
             fl_tot += sflops
             reps += 1
-        line["cpu_baseline"] = {"value": fl_tot / dt_tot / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{reps} x [{desc}]", "seconds": dt_tot}
+        line["cpu_baseline"] = {"value": fl_tot / dt_tot / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": f"{reps} x [{desc}]", "seconds": dt_tot,
+                                "threads": "numpy BLAS (the fp64 attention products) on every core of the "
+                                           "process's affinity set; the quantize/pack/dequant steps are "
+                                           "single-threaded numpy"}
     if dist_ok:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -196,7 +196,15 @@ VARQ_API size_t varq_packed_attention_workspace(const varq_cache_layout* layout,
  *   rope_cos, rope_sin  NULL, or fp32 [T, D/2] tables: pre-RoPE key mode,
  *                key pair (2i, 2i+1) of token t is rotated by (cos, sin)
  *                [t, i] after dequantization ([PAGE] "The block axis",
- *                Eq. 3 and Appendix F).  Both or neither.
+ *                Eq. 3 and Appendix F).  Both or neither; entries are
+ *                cosines and sines (|value| <= 1).  On the tensor cores this
+ *                mode computes S = Q K^T with fp16 operands: every query row
+ *                and the keys of each (batch, head) are first scaled by powers
+ *                of two chosen from the row's largest |q| and from the largest
+ *                |min| + (2^b - 1) scale of the cached key cells, so any bf16
+ *                query and any key within the metadata limits fit fp16 without
+ *                overflow; the scaling is exact and is undone in the softmax
+ *                scale.
  *   out          device bf16 [B, H, lq, D], strides o_sb, o_sh, o_st.
  *   lse          device fp32 [B, H, lq] (natural-log sum of exp of the scaled
  *                scores) or NULL.
@@ -234,13 +242,22 @@ VARQ_API int varq_packed_attention(const varq_cache_layout* layout,
  * GPU that loads it, until the process exits; the caller still passes all
  * inputs and outputs.  Nothing is allocated or freed.
  *   - The first call on a device looks up that array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture begins.  Call with the device that owns `stream` current.
+ *     that device current) and caches it for the life of the process; make
+ *     that first call before any stream capture begins.  Call with the device
+ *     that owns `stream` current.  The cached address belongs to the device's
+ *     current context: do not use this entry point after cudaDeviceReset (or
+ *     anything else that destroys and recreates the primary context) in the
+ *     same process.
  *   - Every call shares the one array: calls whose GPU work overlaps (other
  *     streams, other threads) race.  Serialise them.
- *   - A shape whose partials need more than VARQ_NOALLOC_SCRATCH_BYTES
- *     (varq_packed_attention_workspace(..., VARQ_PATH_SPLIT) tells how much)
- *     returns VARQ_ERR_WORKSPACE before anything is launched.
+ *   - The kernel is chosen as in varq_packed_attention: the CUDA-core kernel
+ *     for lq <= 2 without rope tables, if its partials fit the array, else the
+ *     tensor-core split kernel (fewer ranges, smaller partials).  A shape
+ *     whose partials fit neither returns VARQ_ERR_WORKSPACE before anything is
+ *     launched.  varq_packed_attention_workspace(..., VARQ_PATH_SPLIT) is an
+ *     upper bound of what this call needs: a shape whose query is at most
+ *     VARQ_NOALLOC_SCRATCH_BYTES is always accepted, and one above it may
+ *     still be accepted through the tensor-core kernel.
  */
 #define VARQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 VARQ_API int varq_packed_attention_noalloc(const varq_cache_layout* layout,

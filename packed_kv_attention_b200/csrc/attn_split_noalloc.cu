@@ -14,8 +14,11 @@
 // Host code cannot pass the array's name to a kernel (on the host it is only
 // a stand-in symbol, not a device address), so its device address is looked
 // up once per device with cudaGetSymbolAddress, with that device current, on
-// the first call made on that device, and cached.  That first call should be
-// made before any stream capture begins.
+// the first call made on that device, and cached for the life of the process.
+// That first call should be made before any stream capture begins, and the
+// entry point must not be used after the device's primary context has been
+// destroyed and recreated (cudaDeviceReset): the cached address belongs to the
+// context it was looked up in.
 //
 // All calls share the one array and it keeps whatever the last call left in
 // it.  Nothing needs clearing: every partial the combine kernel reads is
@@ -54,22 +57,8 @@ int scratch_on_current_device(float** out) {
   return VARQ_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool stride_ok(int64_t s) { return (s % 8) == 0; }
-
-int layout_ok(const varq_cache_layout* L) {
-  if (L == nullptr || L->batch < 1 || L->heads < 1) return VARQ_ERR_INVALID_ARG;
-  if (L->head_dim != 64 && L->head_dim != 128) return VARQ_ERR_UNSUPPORTED;
-  if (L->bits < 2 || L->bits > 8 || L->codes_per_word != 32 / L->bits) return VARQ_ERR_INVALID_ARG;
-  if (L->n_blocks < 1 || L->n_blocks > VARQ_MAX_BLOCKS || L->block_start[0] != 0) return VARQ_ERR_INVALID_ARG;
-  for (int i = 0; i < L->n_blocks; ++i)
-    if (L->block_start[i + 1] <= L->block_start[i]) return VARQ_ERR_INVALID_ARG;
-  const int64_t T = L->block_start[L->n_blocks];
-  if (L->n_tokens != T || T > (int64_t(1) << 30)) return VARQ_ERR_INVALID_ARG;
-  if (L->words_per_row != (T + L->codes_per_word - 1) / L->codes_per_word) return VARQ_ERR_INVALID_ARG;
-  if (L->heads > 65535 || L->batch > 65535) return VARQ_ERR_UNSUPPORTED;
-  return VARQ_OK;
-}
+using varq::aligned16;
+using varq::stride_ok;
 
 }  // namespace
 
@@ -78,8 +67,9 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
     const uint32_t* k_packed, const uint32_t* k_meta, const uint32_t* v_packed, const uint32_t* v_meta,
     int n_cached_blocks, float softmax_scale, const float* rope_cos, const float* rope_sin, void* out, int64_t o_sb,
     int64_t o_sh, int64_t o_st, float* lse, uint32_t* dev_status, void* stream) {
-  int rc = layout_ok(L);
+  int rc = varq::check_layout(L);
   if (rc != VARQ_OK) return rc;
+  if (L->heads > 65535 || L->batch > 65535) return VARQ_ERR_UNSUPPORTED;
   if (q == nullptr || out == nullptr || k_packed == nullptr || k_meta == nullptr || v_packed == nullptr ||
       v_meta == nullptr)
     return VARQ_ERR_INVALID_ARG;

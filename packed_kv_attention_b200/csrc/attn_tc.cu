@@ -112,13 +112,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   // Pre-RoPE keys are rotated after dequantization and must be rounded again
   // for the MMA; fp16 (11-bit significand) keeps that rounding 8x below a
-  // bf16 ulp, so S = Q K^T runs in fp16 there (queries convert exactly).
+  // bf16 ulp, so S = Q K^T runs in fp16 there.  Query rows and keys are
+  // scaled by powers of two into fp16 range first (rope_query_exponent,
+  // rope_key_exponent), so queries convert exactly and keys round once.
   constexpr bool QK_F16 = ROPE;
 
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
-  int* sm_bs = reinterpret_cast<int*>(smem + C::OFF_BAR + 512);  // block_start[0..n_cached_blocks]
+  int* sm_bs = reinterpret_cast<int*>(smem + C::OFF_BAR + kBsOffset);  // block_start[0..n_cached_blocks]
+  int8_t* sm_qexp = reinterpret_cast<int8_t*>(smem + C::OFF_BAR + kQexpOffset);  // pre-RoPE: per-row query exponents
   volatile int* abort_flag = &bars->abort_flag;
 
   const int tid = threadIdx.x;
@@ -157,17 +160,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  // query tiles -> K-major swizzled smem (rows past lq are zero)
+  // pre-RoPE key mode: the keys' range from their metadata (fp16 scaling below)
+  if constexpr (ROPE)
+    rope_key_bound_partial<BITS, D, kThreads>(a.k_meta + (int64_t(b) * a.heads + h) * a.n_blocks_total * D,
+                                              a.n_cached_blocks, bars);
+  // query tiles -> K-major swizzled smem (rows past lq are zero).  The CH
+  // chunks of a row are consecutive lanes of one warp in one pass, so with
+  // fp16 operands they agree on the row's exponent by shuffles.
   {
     const __nv_bfloat16* qg = a.q + int64_t(b) * a.q_sb + int64_t(h) * a.q_sh;
     constexpr int CH = D / 8;
-    for (int idx = tid; idx < NQ * BM * CH; idx += kThreads) {
+    constexpr int TOTAL = NQ * BM * CH;
+    static_assert(kThreads % CH == 0, "a row's chunks stay in one warp");
+    for (int base = 0; base < TOTAL; base += kThreads) {
+      const int idx = base + tid;
       const int r = idx / CH, c = idx % CH;
       const int row = qblk * (NQ * BM) + r;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < a.lq) v = __ldg(reinterpret_cast<const uint4*>(qg + int64_t(row) * a.q_st + c * 8));
-      if (QK_F16) v = bf16x8_to_f16x8(v);
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + (r / BM) * C::Q_TILE_BYTES + sw128_offset(r % BM, c * 8, BM)) = v;
+      if (idx < TOTAL && row < a.lq) v = __ldg(reinterpret_cast<const uint4*>(qg + int64_t(row) * a.q_st + c * 8));
+      if constexpr (QK_F16) {
+        uint32_t mb = bf16x8_max_mag(v);
+#pragma unroll
+        for (int o = 1; o < CH; o <<= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        const int qe = rope_query_exponent(mb);
+        v = bf16x8_to_f16x8_scaled(v, exp2i(qe));
+        if (c == 0 && idx < TOTAL) sm_qexp[r] = int8_t(qe);
+      }
+      if (idx < TOTAL)
+        *reinterpret_cast<uint4*>(smem + C::OFF_Q + (r / BM) * C::Q_TILE_BYTES + sw128_offset(r % BM, c * 8, BM)) = v;
     }
     fence_async_smem();
   }
@@ -175,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // pre-RoPE key mode: every key of this (b, h) is scaled by 2^kexp
+  const int kexp = ROPE ? rope_key_exponent_of<kThreads>(bars) : 0;
   // TMEM columns: S of query tile i (double-buffered: buffer j & 1 of KV
   // tile j at 0 or 128) and O_i
   auto s_col = [](int i, int j) -> uint32_t { return C::DB ? uint32_t(j & 1) * 128u : col_s(i); };
@@ -344,9 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint32_t m_cur = tensor == 0 ? mk_cur : mv_cur;
         const uint32_t m_next = tensor == 0 ? mk_next : mv_next;
         const uint32_t* m_glob = tensor == 0 ? mgk : mgv;
+        const float msc = (ROPE && tensor == 0) ? exp2i(kexp) : 1.0f;  // exact: commutes with every rounding below
         auto meta_of = [&](int k) -> float2 {
           const uint32_t w = k == blk_lo ? m_cur : (k == blk_lo + 1 ? m_next : __ldg(m_glob + int64_t(k) * D));
-          return meta_unpack(w);
+          const float2 sm0 = meta_unpack(w);
+          return make_float2(sm0.x * msc, sm0.y * msc);
         };
         float2 sm = meta_of(cb);
         // exact code -> value without a shift per code: the code at bit r of
@@ -435,7 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int r = (warp & 3) * 32 + lane;    // row within the tile == TMEM lane
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
     const uint32_t o_tmem = lane_base + o_col(i);
-    const float sl2 = a.scale_log2;
+    // with fp16 operands the row's query and key scalings are undone here
+    const float sl2 = ROPE ? a.scale_log2 * exp2i(-(int(sm_qexp[i * BM + r]) + kexp)) : a.scale_log2;
     float m_run = -__int_as_float(0x7F800000);
     float l_run = 0.0f;
     bool ok = true;

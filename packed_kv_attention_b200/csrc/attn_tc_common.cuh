@@ -36,8 +36,40 @@ struct Barriers {
   uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
+  uint32_t kmax[20];              // pre-RoPE keys: per-warp largest |min| + (2^b - 1) scale
 };
 static_assert(sizeof(Barriers) <= 512, "the barriers sit below the block-start table");
+
+// Layout of the kBarBytes region: the barriers at 0, the block-start table
+// (VARQ_MAX_BLOCKS + 1 ints) at 512, the per-row query exponents of the
+// pre-RoPE key mode (one int8 per query row of the CTA) at kQexpOffset.
+constexpr uint32_t kBsOffset = 512;
+constexpr uint32_t kQexpOffset = 1552;
+static_assert(kBsOffset + 4 * (VARQ_MAX_BLOCKS + 1) <= kQexpOffset && kQexpOffset + 2 * BM <= kBarBytes,
+              "barrier region layout");
+
+// Largest |min| + (2^b - 1) scale over the key cells of blocks
+// [0, n_cached_blocks) of one (batch, head), reduced over the CTA's threads
+// (one partial per warp in bars->kmax; read after a __syncthreads).
+template <int BITS, int D, int NTHREADS>
+__device__ __forceinline__ void rope_key_bound_partial(const uint32_t* k_meta_bh, int n_cached_blocks,
+                                                       Barriers* bars) {
+  const float qmax = float((1u << BITS) - 1u);
+  uint32_t mb = 0;
+  for (int i = threadIdx.x; i < n_cached_blocks * D; i += NTHREADS) {
+    const float2 sm = meta_unpack(__ldg(k_meta_bh + i));
+    mb = max(mb, __float_as_uint(fabsf(sm.y) + qmax * fabsf(sm.x)));
+  }
+  mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+  if ((threadIdx.x & 31) == 0) bars->kmax[threadIdx.x >> 5] = mb;
+}
+template <int NTHREADS>
+__device__ __forceinline__ int rope_key_exponent_of(const Barriers* bars) {
+  uint32_t mb = 0;
+#pragma unroll
+  for (int w = 0; w < NTHREADS / 32; ++w) mb = max(mb, bars->kmax[w]);
+  return rope_key_exponent(mb);
+}
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const bool ok = mbar_wait(bar, parity, abort_flag);

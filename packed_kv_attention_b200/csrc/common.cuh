@@ -401,13 +401,50 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 8 bf16 (one 16-byte chunk) -> 8 fp16; exact for |x| in [2^-14, 65504].
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+// 2^n as fp32, exact, for n in [-126, 127].
+__device__ __forceinline__ float exp2i(int n) { return __int_as_float((n + 127) << 23); }
+
+// 8 bf16 (one 16-byte chunk) times a power of two f -> 8 fp16.  The product is
+// exact; the conversion is exact wherever x f lies in [2^-14, 65504].
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_scaled(uint4 v, float f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = pack_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  for (int i = 0; i < 4; ++i)
+    o[i] = pack_f16x2(__uint_as_float(w[i] << 16) * f, __uint_as_float(w[i] & 0xFFFF0000u) * f);
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Largest magnitude bit pattern (sign dropped) of the 8 bf16 of a chunk; for
+// finite values the order of these patterns is the order of |x|.
+__device__ __forceinline__ uint32_t bf16x8_max_mag(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  return m;
+}
+
+// Pre-RoPE key mode: S = Q K^T runs in fp16, whose range ends at 65504, while
+// queries are any bf16 and a dequantized key reaches |min| + (2^b - 1) scale
+// (up to ~1.7e7 inside the metadata limits), rotated by up to sqrt(2).  Each
+// query row is scaled by 2^qe and every key of a (batch, head) by 2^ke, both
+// chosen so the largest value stays below 2^15; the scaling is exact and the
+// softmax scale of a row is multiplied by 2^-(qe + ke), also exactly, so the
+// scores are the unscaled ones up to the same fp16 roundings (half an ulp
+// relative) as in range.
+// Query row whose largest magnitude pattern is mb (bf16 bits without sign).
+__device__ __forceinline__ int rope_query_exponent(uint32_t mb) {
+  if (mb == 0) return 0;
+  const int e = int(mb >> 7) - 127;  // the largest |q| lies in [2^e, 2^(e+1))
+  return min(60, max(-60, 14 - e));
+}
+// Keys whose largest |min| + (2^b - 1) scale over the cached cells has fp32
+// bit pattern mb: |rotated key| < 2^(e+1) (1 + 2^-8) sqrt(2) < 2^(e+1.51).
+__device__ __forceinline__ int rope_key_exponent(uint32_t mb) {
+  if (mb == 0) return 0;
+  const int e = int((mb >> 23) & 0xFFu) - 127;
+  return min(60, max(-60, 13 - e));
 }
 
 // Packed pairs of fp32 (sm_100): one instruction applies an IEEE fp32

@@ -11,6 +11,31 @@
 
 namespace varq {
 
+// ------------------------------------------------- argument checks (host)
+
+// The checks every entry point applies to its pointers, strides and cache
+// layout before anything is launched (one definition for all of them).
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool stride_ok(int64_t s) { return (s % 8) == 0; }
+constexpr int64_t kMaxTokens = int64_t(1) << 30;
+// VARQ_OK, or the status a malformed or unsupported layout returns.
+inline int check_layout(const varq_cache_layout* L) {
+  if (L == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (L->batch < 1 || L->heads < 1) return VARQ_ERR_INVALID_ARG;
+  if (L->head_dim != 64 && L->head_dim != 128) return VARQ_ERR_UNSUPPORTED;
+  if (L->bits < 2 || L->bits > 8) return VARQ_ERR_INVALID_ARG;
+  if (L->codes_per_word != 32 / L->bits) return VARQ_ERR_INVALID_ARG;
+  if (L->n_blocks < 1 || L->n_blocks > VARQ_MAX_BLOCKS) return VARQ_ERR_INVALID_ARG;
+  if (L->block_start[0] != 0) return VARQ_ERR_INVALID_ARG;
+  for (int i = 0; i < L->n_blocks; ++i)
+    if (L->block_start[i + 1] <= L->block_start[i]) return VARQ_ERR_INVALID_ARG;
+  const int64_t T = L->block_start[L->n_blocks];
+  if (L->n_tokens != T || T > kMaxTokens) return VARQ_ERR_INVALID_ARG;
+  const int64_t W = (T + L->codes_per_word - 1) / L->codes_per_word;
+  if (L->words_per_row != W) return VARQ_ERR_INVALID_ARG;
+  return VARQ_OK;
+}
+
 // ---------------------------------------------------------- quantize+pack
 
 struct QuantArgs {

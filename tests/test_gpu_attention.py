@@ -171,6 +171,31 @@ def test_attention_pre_rope_keys(path, lq, D):
         _check(out, lse, ref, ref_lse, 0, h, rows)
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("path,lq", [(V.PATH_TENSOR, 200), (V.PATH_SPLIT, 8)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_pre_rope_beyond_fp16_range(bits, path, lq, D):
+    """Pre-RoPE keys whose cells reach 9e4 (INT2) to 4e5 (INT4) while staying
+    inside the metadata limits (min >= 0, scale <= 65504), and queries up to
+    ~6e5: both beyond the fp16 range in which S = Q K^T runs in this mode.  A
+    custom softmax scale keeps the scores moderate.  The tensor path (pair of CTAs)
+    and the split-KV form must match the fp64 oracle with no status bit set."""
+    sizes = [120, 120, 120, 45]
+    bs = synth.block_starts(sizes)
+    k, v, q, cos, sin = _inputs(1, 2, D, sizes, lq, seed=17 + bits, rope=True)
+    k = (k.float().abs() * 2.0 ** (11 if bits == 4 else 9)).to(torch.bfloat16)  # powers of two: exact
+    q = (q.float() * 2.0 ** 17).to(torch.bfloat16)
+    scale = 2.0 ** -28 / math.sqrt(D) * (4.0 if bits == 2 else 1.0)
+    assert float(k.float().abs().max()) > 65504 and float(q.float().abs().max()) > 65504
+    L = V.varq_cache_alloc(1, 2, D, bits, bs)
+    out, lse = _gpu_attention(L, k, v, q, len(sizes), cos=cos, sin=sin, path=path, scale=scale)
+    assert bool(torch.isfinite(out.float()).all())
+    rows = np.arange(lq)
+    for h in range(2):
+        ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), 0, h, rows, cos=cos, sin=sin, scale=scale)
+        _check(out, lse, ref, ref_lse, 0, h, rows)
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("lq", [1, 2])

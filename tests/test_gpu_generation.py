@@ -110,3 +110,32 @@ def test_generation_loop_captures_in_a_cuda_graph():
     for o, e in zip(outs, eager):
         assert torch.equal(o, e)
     assert loop.device_status() == 0
+
+
+@pytest.mark.parametrize("frame_tokens", [1560, 4680])
+def test_generation_loop_next_frame_grouping(frame_tokens):
+    """Next-frame generation with pre-RoPE keys, grouped per latent frame of
+    1,560 tokens (the README's default grouping unit) or per chunk of three
+    frames (4,680 tokens, the workloads' grouping): nine frames appended one
+    group at a time, each group's queries (sampled rows, including tile edges)
+    attending to every group so far, against the oracle."""
+    bits, D, B, H = 4, 128, 1, 2
+    n_frames = 9
+    sizes = [frame_tokens] * (n_frames * 1560 // frame_tokens)
+    g, k, v = _cache(31, B, H, sizes, D)
+    bs = synth.block_starts(sizes)
+    cos, sin = synth.rope_tables_3d(bs[-1], D)
+    loop = PackedKVLoop(B, H, D, bits, sizes, device=DEV)
+    kd, vd, cd, sd = k.to(DEV), v.to(DEV), cos.to(DEV), sin.to(DEV)
+    rng = np.random.default_rng(frame_tokens)
+    for step, n in enumerate(sizes):
+        q = synth.queries(g, B, H, n, D)
+        lse = torch.empty(B, H, n, dtype=torch.float32, device=DEV)
+        out = loop.step(step, kd[:, :, bs[step]:bs[step + 1]], vd[:, :, bs[step]:bs[step + 1]], q.to(DEV), lse=lse,
+                        rope_cos=cd, rope_sin=sd)
+        torch.cuda.synchronize()
+        rows = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.integers(0, n, 12)]))
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k, v, q, bs, bits, step + 1, 0, h, rows, cos=cos, sin=sin)
+            _check(out, lse, ref, ref_lse, 0, h, rows)
+    assert loop.device_status() == 0
