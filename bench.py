@@ -377,7 +377,7 @@ def measure_rows(dev, stream, peaks, iters=5):
     vp4, vm4 = V.alloc_cache(L4, dev)
     V.varq_quantize_pack(L4, v, vp4, vm4, dev_status=st, stream=stream)
     split = {}
-    for lq in (1, 16):
+    for lq in (1, 4, 16):
         q = data["q"][:, :, :lq].contiguous()
         o = torch.empty_like(q)
         ws_bytes = V.varq_packed_attention_workspace(L4, lq, w.n_blocks, V.PATH_SPLIT)
@@ -511,6 +511,182 @@ def measure_rows(dev, stream, peaks, iters=5):
     return rows
 
 
+def _median_ms(fn, stream, iters, warm=2):
+    for _ in range(warm):
+        fn()
+    return statistics.median(_event_times(fn, stream, iters))
+
+
+def roofline_frac(flops, nbytes, ms, peaks):
+    """Binding roofline time (tensor at the burst bf16 peak, or HBM) over the
+    measured time, and which one binds."""
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    return max(t_tc, t_hbm) / (ms * 1e-3), ("tensor" if t_tc >= t_hbm else "hbm")
+
+
+def measure_fused_vs_unfused(dev, stream, peaks, bits=4, iters=3):
+    """Kernel-sweep cache (B8 H32 T16384 D128, 16 blocks of 1,024), query
+    blocks of 1 to 4,096 tokens: the fused packed-KV attention against the
+    unfused baseline (unpack+dequant of K and V into dense bf16, then dense
+    tensor-core attention over them), each against its binding roofline."""
+    from packed_kv_attention_b200 import varq as V
+    w = synth.WORKLOADS["sweep"]
+    data = synth.make_inputs(w, lq=max(w.lq), seed=6, device=dev)
+    bs = data["block_start"]
+    L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, bs)
+    kp, km = V.alloc_cache(L, dev)
+    vp, vm = V.alloc_cache(L, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    V.varq_quantize_pack(L, data["k"], kp, km, dev_status=st, stream=stream)
+    V.varq_quantize_pack(L, data["v"], vp, vm, dev_status=st, stream=stream)
+    kd, vd = data["k"], data["v"]  # reused as the dense workspaces (overwritten by unpack+dequant)
+    torch.cuda.synchronize()
+    T, B, H, D = w.n_tokens, w.batch, w.heads, w.head_dim
+    dense_bytes = B * H * T * D * 2
+    out = {}
+    for lq in w.lq:
+        q = data["q"][:, :, :lq].contiguous()
+        o = torch.empty_like(q)
+        ws_f = V.varq_packed_attention_workspace(L, lq, w.n_blocks)
+        wsf = torch.empty(max(ws_f // 4, 1), dtype=torch.float32, device=dev)
+        ws_d = V.varq_dense_attention_workspace(B, H, D, lq, T)
+        wsd = torch.empty(max(ws_d // 4, 1), dtype=torch.float32, device=dev)
+
+        def fused():
+            V.varq_packed_attention(L, q, kp, km, vp, vm, o, workspace=wsf, dev_status=st, stream=stream)
+
+        def unpack():
+            V.varq_unpack_dequant(L, kp, km, kd, stream=stream)
+            V.varq_unpack_dequant(L, vp, vm, vd, stream=stream)
+
+        def dense():
+            V.varq_dense_attention(q, kd, vd, o, workspace=wsd, dev_status=st, stream=stream)
+
+        def unfused():
+            unpack()
+            dense()
+        t_f = _median_ms(fused, stream, iters)
+        t_u = _median_ms(unfused, stream, iters)
+        t_up = _median_ms(unpack, stream, iters)
+        t_d = _median_ms(dense, stream, iters)
+        fl = attention_flops(w, lq)
+        b_f = attention_bytes(L, w, lq, False)
+        # unfused bytes: unpack reads the packed cache and writes dense K, V;
+        # the dense attention reads them back (plus Q, O)
+        b_up = 2 * (L.packed_bytes + L.meta_bytes + dense_bytes)
+        b_d = 2 * B * H * lq * D * 2 + 2 * dense_bytes
+        fr_f, bound_f = roofline_frac(fl, b_f, t_f, peaks)
+        fr_u, bound_u = roofline_frac(fl, b_up + b_d, t_u, peaks)
+        fr_d, bound_d = roofline_frac(fl, b_d, t_d, peaks)
+        out[f"lq{lq}"] = {
+            "fused_us": 1e3 * t_f, "fused_TFLOP/s": fl / (t_f * 1e-3) / 1e12, "fused_bound": bound_f,
+            "fused_frac": fr_f,
+            "unfused_us": 1e3 * t_u, "unfused_unpack_us": 1e3 * t_up, "unfused_dense_attention_us": 1e3 * t_d,
+            "unfused_frac": fr_u, "unfused_bound": bound_u, "dense_attention_frac": fr_d,
+            "dense_attention_bound": bound_d, "fused_speedup": t_u / t_f}
+        del q, o, wsf, wsd
+    res = {"workload": f"sweep: B={B} H={H} D={D} T={T} blocks={w.n_blocks} INT{bits}; fused = "
+                       "varq_packed_attention (AUTO path), unfused = varq_unpack_dequant of K and V into dense bf16 + "
+                       "varq_dense_attention; fractions of the binding roofline (burst bf16 peak or HBM) over each "
+                       "path's own algorithmic bytes", **out, "device_status": int(st.item())}
+    del data, kp, km, vp, vm, kd, vd
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_longlive(dev, stream, peaks, iters=3):
+    """LongLive-like long-horizon layer (B4 H12 D128, 40 chunks of 4,680
+    tokens = 187,200 cached, pre-RoPE keys rotated after dequantization, one
+    4,680-token query block) at INT2, INT3 and INT4: quantize+pack of K and V
+    and the fused attention, each against its roofline."""
+    from packed_kv_attention_b200 import varq as V
+    w = synth.WORKLOADS["longlive"]
+    data = synth.make_inputs(w, lq=w.lq[-1], seed=7, device=dev)
+    bs = data["block_start"]
+    cos, sin = data["rope_cos"], data["rope_sin"]
+    lq = w.lq[-1]
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    o = torch.empty_like(data["q"])
+    res = {}
+    for bits in w.bits:
+        L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, bs)
+        kp, km = V.alloc_cache(L, dev)
+        vp, vm = V.alloc_cache(L, dev)
+
+        def quant():
+            V.varq_quantize_pack(L, data["k"], kp, km, dev_status=st, stream=stream)
+            V.varq_quantize_pack(L, data["v"], vp, vm, dev_status=st, stream=stream)
+
+        def attn():
+            V.varq_packed_attention(L, data["q"], kp, km, vp, vm, o, rope_cos=cos, rope_sin=sin, dev_status=st,
+                                    stream=stream)
+        t_q = _median_ms(quant, stream, iters)
+        t_a = _median_ms(attn, stream, iters)
+        fl = attention_flops(w, lq)
+        qb = quant_bytes(L, w)
+        ab = attention_bytes(L, w, lq, True)
+        fr_a, bound = roofline_frac(fl, ab, t_a, peaks)
+        res[f"int{bits}"] = {"quant_pack_us": 1e3 * t_q, "quant_pack_GB/s": qb / (t_q * 1e-3) / 1e9,
+                             "quant_pack_frac_hbm": qb / (t_q * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "attention_ms": t_a, "attention_TFLOP/s": fl / (t_a * 1e-3) / 1e12,
+                             "attention_bound": bound, "attention_frac": fr_a,
+                             "attention_frac_sustained": fl / (t_a * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        del kp, km, vp, vm
+    res = {"workload": f"longlive: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} blocks={w.n_blocks} "
+                       f"Lq={lq} pre-RoPE keys (3D RoPE tables)", **res, "device_status": int(st.item())}
+    del data, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_var_d16(dev, stream, peaks, iters=20):
+    """VAR-d16-like layer as one call each (B1 H16 D64, 10 scales = 680 tokens,
+    INT4, the last 256-token block attending to all 680): quantize+pack of K
+    and V and the attention, captured once in a CUDA graph and replayed (at
+    these sizes the launch costs dominate; the roofline time is below a
+    microsecond)."""
+    from packed_kv_attention_b200 import varq as V
+    w = synth.WORKLOADS["var_d16"]
+    pipe = Pipeline(w, 4, w.lq[-1], dev, seed=8)
+    torch.cuda.synchronize()
+
+    def step():
+        pipe.step(stream)
+
+    def attn():
+        V.varq_packed_attention(pipe.L, pipe.q, pipe.kp, pipe.km, pipe.vp, pipe.vm, pipe.out, workspace=pipe.ws,
+                                dev_status=pipe.status, stream=stream)
+    res = {}
+    for name, fn in (("step", step), ("attention", attn)):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+
+        def replay():
+            with torch.cuda.stream(stream):
+                g.replay()
+        t_graph = _median_ms(replay, stream, iters, warm=3)
+        t_launch = _median_ms(fn, stream, iters, warm=3)
+        res[name] = {"graph_replay_us": 1e3 * t_graph, "stream_launched_us": 1e3 * t_launch}
+        del g
+    fl = attention_flops(w, w.lq[-1])
+    fr, bound = roofline_frac(fl, attention_bytes(pipe.L, w, w.lq[-1], False), res["attention"]["graph_replay_us"] * 1e-3,
+                              peaks)
+    res["attention"].update({"TFLOP/s": fl / (res["attention"]["graph_replay_us"] * 1e-6) / 1e12, "bound": bound,
+                             "frac": fr})
+    res["step"]["launches"] = pipe.launches_per_step
+    out = {"workload": f"var_d16: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} blocks={w.n_blocks} "
+                       f"Lq={w.lq[-1]} INT4; one step = quantize+pack K, V + attention", **res,
+           "device_status": int(pipe.status.item())}
+    del pipe
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_of(w, args):
     return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} "
                         f"blocks={w.n_blocks} Lq={args.lq} INT{args.bits}",
@@ -629,6 +805,9 @@ def main(argv=None):
         del pipe
         torch.cuda.empty_cache()
         line["rows"] = measure_rows(dev, stream, peaks)
+        line["rows"]["c5_fused_vs_unfused"] = measure_fused_vs_unfused(dev, stream, peaks)
+        line["rows"]["c4_longlive"] = measure_longlive(dev, stream, peaks)
+        line["rows"]["c1_var_d16"] = measure_var_d16(dev, stream, peaks)
         pipe = Pipeline(w, args.bits, args.lq, dev)
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(pipe, max(3, args.steps // 2), 2, stream)

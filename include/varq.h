@@ -269,6 +269,44 @@ VARQ_API int varq_packed_attention_noalloc(const varq_cache_layout* layout,
                                            void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
                                            float* lse, uint32_t* dev_status, void* stream);
 
+/*
+ * varq_dense_attention_workspace -- bytes of device workspace
+ * varq_dense_attention needs for this shape and path (0 if none: the tensor
+ * path, or invalid arguments).
+ */
+VARQ_API size_t varq_dense_attention_workspace(int batch, int heads, int head_dim, int lq, int64_t n_tokens,
+                                               int path);
+
+/*
+ * varq_dense_attention -- O = softmax(scale * Q K^T) V over dense bf16 K and V:
+ * the attention half of the unfused baseline, which first expands the packed
+ * cache into dense bf16 workspaces with varq_unpack_dequant and then attends
+ * over them ([README] "Fused-kernel overhead reduction": the fused kernel is
+ * compared against that unfused runtime; "Memory-Efficient Runtime": the dense
+ * dequantization workspaces it needs).  Tensor cores (tcgen05) with K and V
+ * tiles loaded by the TMA engine.
+ *
+ *   batch, heads, head_dim (64 or 128), n_tokens   K and V hold n_tokens
+ *                attended tokens per (batch, head).
+ *   q            device bf16 [B, H, lq, D], strides q_sb, q_sh, q_st.
+ *   k, v         device bf16 [B, H, n_tokens, D], element strides
+ *                (k_sb, k_sh, k_st), (v_sb, v_sh, v_st); channels contiguous.
+ *   out, lse, softmax_scale, workspace, path, dev_status   as in
+ *                varq_packed_attention (workspace from
+ *                varq_dense_attention_workspace; SPLIT needs lq <=
+ *                VARQ_SPLIT_MAX_LQ).
+ * Pointers 16-byte aligned, strides multiples of 8 elements.  Returns
+ * VARQ_ERR_UNSUPPORTED when the driver cannot build a TMA descriptor for the
+ * given strides.
+ */
+VARQ_API int varq_dense_attention(int batch, int heads, int head_dim, int64_t n_tokens,
+                                  const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st, int lq,
+                                  const void* k, int64_t k_sb, int64_t k_sh, int64_t k_st,
+                                  const void* v, int64_t v_sb, int64_t v_sh, int64_t v_st,
+                                  float softmax_scale, void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
+                                  float* lse, void* workspace, size_t workspace_bytes, int path,
+                                  uint32_t* dev_status, void* stream);
+
 /* Human-readable name of a varq_status value (static string). */
 VARQ_API const char* varq_status_string(int status);
 

@@ -199,8 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int kexp = ROPE ? rope_key_exponent_of<kThreads>(bars) : 0;
   // TMEM columns: S of query tile i (double-buffered: buffer j & 1 of KV
   // tile j at 0 or 128) and O_i
-  auto s_col = [](int i, int j) -> uint32_t { return C::DB ? uint32_t(j & 1) * 128u : col_s(i); };
-  auto o_col = [](int i) -> uint32_t { return C::DB ? 256u : col_o<NQ>(i); };
+  auto s_col = [](int i, int j) -> uint32_t { return s_col_of<NQ, C::DB>(i, j); };
+  auto o_col = [](int i) -> uint32_t { return o_col_of<NQ, C::DB>(i); };
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -221,9 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         bulk_g2s(sb + C::WORDS_BYTES, vw + int64_t(w0) * D, wbytes, &bars->full[st]);
         issued = j + 1;
       }
-      // never leave copies in flight: wait for every stage that was filled
-      for (int j = max(0, issued - C::PST); j < issued; ++j)
-        mbar_wait(&bars->full[j % C::PST], (j / C::PST) & 1, abort_flag);
+      // never leave copies in flight, even after an abort: wait for every
+      // stage that was filled
+      for (int j = max(0, issued - C::PST); j < issued; ++j) mbar_wait_drain(&bars->full[j % C::PST], (j / C::PST) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
@@ -256,71 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           mma_ts(tmem + o_col(i), tmem + s_col(i, j) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      if constexpr (C::DB) {
-        // one query tile: S(0), S(1) first, then per KV tile j PV(j) and S(j + 2)
-        // into the buffer P(j) is read from (the MMAs run in issue order);
-        // barriers indexed by j & 1
-        bool ok = true;
-        for (int j = 0; j < min(2, ntiles) && ok; ++j) {
-          ok = mbar_wait(&bars->kready[j % C::KST], (j / C::KST) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, j);
-          mma_commit(&bars->s_full[j & 1]);
-          mma_commit(&bars->kfree[j % C::KST]);
-        }
-        for (int j = 0; j < ntiles && ok; ++j) {
-          ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag) &&
-               mbar_wait(&bars->p_ready[j & 1], (j >> 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(0, j);
-          mma_commit(&bars->o_done[j & 1]);
-          mma_commit(&bars->vfree[j % C::VST]);
-          if (j + 2 < ntiles) {
-            ok = mbar_wait(&bars->kready[(j + 2) % C::KST], ((j + 2) / C::KST) & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_qk(0, j + 2);
-            mma_commit(&bars->s_full[j & 1]);
-            mma_commit(&bars->kfree[(j + 2) % C::KST]);
-          }
-        }
-      } else {
-        bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, abort_flag);
-        if (ok) {
-          tc_fence_after();
-          for (int i = 0; i < NQ; ++i) {
-            issue_qk(i, 0);
-            mma_commit(&bars->s_full[i]);
-          }
-          mma_commit(&bars->kfree[0]);
-        }
-        for (int j = 0; j < ntiles && ok; ++j) {
-          ok = mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag);
-          for (int i = 0; i < NQ && ok; ++i) {
-            ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(i, j);
-            mma_commit(&bars->o_done[i]);
-            if (i == NQ - 1) mma_commit(&bars->vfree[j % C::VST]);
-            if (j + 1 < ntiles) {
-              if (i == 0) {
-                ok = mbar_wait(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-              }
-              issue_qk(i, j + 1);
-              mma_commit(&bars->s_full[i]);
-              if (i == NQ - 1) mma_commit(&bars->kfree[(j + 1) % C::KST]);
-            }
-          }
-        }
-      }
-      // every MMA issued so far has finished before TMEM is released
-      mma_commit(&bars->teardown);
-      mbar_wait(&bars->teardown, 0, abort_flag);
+      mma_issue_loop<NQ, C::DB, C::KST, C::VST>(bars, ntiles, issue_qk, issue_pv);
     }
   } else if (warp >= kDequantWarp0 || (NQ == 1 && warp >= 4)) {
     // ------------------------------------------------------------- dequant
@@ -455,206 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else if ((warp >> 2) < NQ) {
     // ------------------------------------------------------------- softmax
-    const int i = warp >> 2;                 // query tile of this warpgroup
-    const int r = (warp & 3) * 32 + lane;    // row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
-    const uint32_t o_tmem = lane_base + o_col(i);
+    const int i = warp >> 2, r = (warp & 3) * 32 + lane;
     // with fp16 operands the row's query and key scalings are undone here
     const float sl2 = ROPE ? a.scale_log2 * exp2i(-(int(sm_qexp[i * BM + r]) + kexp)) : a.scale_log2;
-    float m_run = -__int_as_float(0x7F800000);
-    float l_run = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      // S of this tile: TMEM columns and barrier (buffer j & 1 when double-buffered)
-      const uint32_t s_tmem = lane_base + s_col(i, j);
-      ok = C::DB ? wait_all(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag)
-                 : wait_all(&bars->s_full[i], j & 1, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      const int valid = min(C::NKV, t_att - (tile0 + j) * C::NKV);
-      // pass 1: row maximum of the raw scores
-      float mx = -__int_as_float(0x7F800000);
-#pragma unroll
-      for (int c0 = 0; c0 < C::NKV; c0 += 32) {
-        if (c0 + 32 <= C::NKV) {
-          uint32_t v[32];
-          tmem_ld32(s_tmem + c0, v);
-          tmem_wait_ld_dep(v);
-          if (valid == C::NKV) {
-            float m2 = mx;
-#pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              mx = fmax3(mx, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
-              m2 = fmax3(m2, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
-            }
-            mx = fmaxf(mx, m2);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (c0 + k < valid) mx = fmaxf(mx, __uint_as_float(v[k]));
-          }
-        } else {
-          uint32_t v[16];
-          tmem_ld16(s_tmem + c0, v);
-          tmem_wait_ld_dep16(v);
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (c0 + k < valid) mx = fmaxf(mx, __uint_as_float(v[k]));
-        }
-      }
-      mx *= sl2;
-      float m_new = m_run;
-      if (j == 0 || mx > m_run + kRescaleThreshold) m_new = fmaxf(mx, m_run);
-      const float alpha = (j == 0) ? 0.0f : ex2_approx(m_run - m_new);
-      // PV_i of the previous tile has finished before O_i is rescaled.  With S
-      // double-buffered, o_done[t & 1] completes once per PV(t) of that
-      // parity; a wait names tile t's phase, exact while tile t - 2's has been
-      // waited for and PV(t + 2) cannot have run: PV(j - 2) is waited for every
-      // tile (long finished), PV(j - 1) only to rescale O.
-      if (C::DB && j >= 2) {
-        ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag);
-        if (!ok) break;
-      }
-      if (j >= 1 && (!C::DB || __any_sync(0xFFFFFFFFu, m_new != m_run))) {
-        ok = C::DB ? wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)
-                   : wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xFFFFFFFFu, m_new != m_run)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(o_tmem + c0, v);
-            tmem_wait_ld_dep(v);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-            tmem_st32(o_tmem + c0, v);
-          }
-        }
-      }
-      // pass 2: P = exp2(S * scale_log2 - m_new) as bf16 pairs over the consumed S columns
-      const float neg_m = -m_new;
-      const uint64_t sl2p = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
-      uint64_t rs2 = f2_pack(0.0f, 0.0f);
-      float rs = 0.0f;
-#pragma unroll
-      for (int c0 = 0; c0 < C::NKV; c0 += 32) {
-        if (c0 + 32 <= C::NKV) {
-          uint32_t v[32];
-          tmem_ld32(s_tmem + c0, v);
-          tmem_wait_ld_dep(v);
-          uint32_t pk[16];
-          if (valid == C::NKV) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              float t0, t1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), sl2p, negm2), t0,
-                        t1);
-              const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-              rs2 = f2_add(rs2, f2_pack(p0, p1));
-              pk[k] = pack_bf16x2(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
-              float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
-              p0 = (c0 + 2 * k < valid) ? p0 : 0.0f;
-              p1 = (c0 + 2 * k + 1 < valid) ? p1 : 0.0f;
-              rs += p0 + p1;
-              pk[k] = pack_bf16x2(p0, p1);
-            }
-          }
-          tmem_st16(s_tmem + c0 / 2, pk);
-        } else {
-          uint32_t v[16];
-          tmem_ld16(s_tmem + c0, v);
-          tmem_wait_ld_dep16(v);
-          uint32_t pk[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k]), sl2, neg_m));
-            float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[2 * k + 1]), sl2, neg_m));
-            p0 = (c0 + 2 * k < valid) ? p0 : 0.0f;
-            p1 = (c0 + 2 * k + 1 < valid) ? p1 : 0.0f;
-            rs += p0 + p1;
-            pk[k] = pack_bf16x2(p0, p1);
-          }
-          tmem_st8(s_tmem + c0 / 2, pk);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(C::DB ? &bars->p_ready[j & 1] : &bars->p_ready[i]);
-      {
-        float r0, r1;
-        f2_unpack(rs2, r0, r1);
-        rs += r0 + r1;
-      }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-    }
-    // ------------------------------------------------------------- epilogue
-    // O_i is final once the last PV_i has completed (double-buffered S: PV of
-    // the last two tiles, waited for in order)
-    auto o_final = [&]() {
-      if constexpr (C::DB) {
-        return (ntiles < 2 || wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, abort_flag)) &&
-               wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag);
-      } else {
-        return wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
-      }
-    };
-    if (a.kv_split) {
-      // split-KV form: the unnormalised partial of this KV range (O, running
-      // max m in the log2 domain, running sum l); m = -inf marks "no token"
-      const int row = qblk * (NQ * BM) + i * BM + r;
-      float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
-                  int64_t(row) * (D + 2);
-      const bool have = ok && ntiles > 0 && o_final();
-      if (have) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(o_tmem + c0, v);
-          tmem_wait_ld_dep(v);
-          if (row < a.lq) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              *reinterpret_cast<float2*>(ws + c0 + 2 * k) =
-                  make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-          }
-        }
-      }
-      if (row < a.lq) {
-        ws[D] = have ? m_run : -__int_as_float(0x7F800000);
-        ws[D + 1] = have ? l_run : 0.0f;
-      }
-    } else if (ok && ntiles > 0 && o_final()) {
-      tc_fence_after();
-      const int row = qblk * (NQ * BM) + i * BM + r;
-      const float inv = 1.0f / l_run;
-      __nv_bfloat16* og = a.out + int64_t(b) * a.o_sb + int64_t(h) * a.o_sh + int64_t(row) * a.o_st;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(o_tmem + c0, v);
-        tmem_wait_ld_dep(v);
-        if (row < a.lq) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              pk[k] = pack_bf16x2(__uint_as_float(v[c * 8 + 2 * k]) * inv, __uint_as_float(v[c * 8 + 2 * k + 1]) * inv);
-            *reinterpret_cast<uint4*>(og + c0 + c * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      }
-      if (row < a.lq && a.lse != nullptr)
-        a.lse[(int64_t(b) * a.heads + h) * a.lq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-    }
+    softmax_loop<C::NKV, D, NQ, C::DB>(a, bars, tmem, warp, lane, qblk, split, b, h, tile0, ntiles, sl2);
   }
 
   // ------------------------------------------------------------- teardown

@@ -214,9 +214,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           bulk_g2s(sb + C::WORDS_K + i * vrow, vw + int64_t(w0 + i) * D + int(rank) * C::DH, vrow, &bars->full[st]);
         issued = j + 1;
       }
-      // never leave copies in flight: wait for every stage that was filled
-      for (int j = max(0, issued - C::PST); j < issued; ++j)
-        mbar_wait(&bars->full[j % C::PST], (j / C::PST) & 1, abort_flag);
+      // never leave copies in flight, even after an abort: wait for every
+      // stage that was filled
+      for (int j = max(0, issued - C::PST); j < issued; ++j) mbar_wait_drain(&bars->full[j % C::PST], (j / C::PST) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
@@ -279,9 +279,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           }
         }
       }
-      // every MMA issued so far has finished before TMEM is released
+      // every MMA issued so far has finished before TMEM is released (also
+      // after an abort: the drain waits for this thread's own MMAs only)
       mma2_commit_both(&bars->teardown);
-      mbar_wait(&bars->teardown, 0, abort_flag);
+      mbar_wait_drain(&bars->teardown, 0);
     } else if (lane == 0) {
       // rank 1: relay P(j) of each query tile to rank 0, then keep TMEM until
       // the pair's MMAs have finished
@@ -291,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
           if (ok) mbar_arrive_rank(&bars->p_ready[i], 0);
         }
-      mbar_wait(&bars->teardown, 0, abort_flag);
+      mbar_wait_drain(&bars->teardown, 0);
     }
   } else if (warp == kRelayWarp) {
     // ------------------------------------------------------------- relay

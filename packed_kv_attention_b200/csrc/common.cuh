@@ -103,6 +103,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait for a phase that completes without any other thread's help: bulk
+// copies or MMAs this thread has already issued.  The abort flag is ignored
+// (after an abort the CTA must still not exit, or free TMEM, with its own
+// copies or MMAs in flight); the wait is bounded like every other.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_suspend(a, parity, kSuspendHintNs)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_suspend(a, parity, kSuspendHintNs)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // ------------------------------------------------- thread-block clusters
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -157,6 +171,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Tiled TMA load of one box of a 4-D tensor map (a __grid_constant__ kernel
+// parameter, passed by its generic address) into shared memory, completion
+// counted on `bar` in bytes.  The innermost coordinate times the element size
+// must be a multiple of 16 bytes; elements outside the tensor read as zero.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -102,6 +102,13 @@ struct AttnArgs {
   int32_t block_start[VARQ_MAX_BLOCKS + 1];
 };
 
+// A dense bf16 [B, H, T, D] tensor: base pointer and element strides
+// (channels contiguous).
+struct DenseTensor {
+  const void* ptr;
+  int64_t sb, sh, st;
+};
+
 // Tensor-core attention; with kv_split, the split-KV form plus its combine.
 // Pre-RoPE keys on the tensor path go to the paired-CTA kernel
 // (launch_attention_tc2), everything else to the single-CTA one.
@@ -119,5 +126,12 @@ constexpr int kDecodeMaxLq = 2;
 bool use_decode_kernel(const AttnArgs& a);
 int split_kv_decode_splits(const AttnArgs& a);
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
+// Attention over dense bf16 K and V (the unfused baseline's second half), on
+// the tensor cores with TMA-loaded tiles; with kv_split, the split-KV form plus
+// the combine.  Returns a varq_status (VARQ_ERR_UNSUPPORTED when a tensor map
+// cannot describe the strides).
+int launch_attention_dense(const AttnArgs& a, const DenseTensor& k, const DenseTensor& v, cudaStream_t stream);
+// Number of KV ranges of the dense kernel's split-KV form.
+int dense_splits(const AttnArgs& a);
 
 }  // namespace varq

@@ -227,4 +227,69 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   return launch_status(dec ? varq::launch_attention_decode(a, s) : varq::launch_attention_tc(a, s));
 }
 
+static int check_dense(int batch, int heads, int head_dim, int64_t n_tokens, int lq, int path) {
+  if (batch < 1 || heads < 1 || lq < 1 || n_tokens < 1) return VARQ_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return VARQ_ERR_UNSUPPORTED;
+  if (n_tokens > kMaxTokens || batch > 65535 || heads > 65535) return VARQ_ERR_UNSUPPORTED;
+  if (path != VARQ_PATH_AUTO && path != VARQ_PATH_TENSOR && path != VARQ_PATH_SPLIT) return VARQ_ERR_INVALID_ARG;
+  if (choose_path(lq, path) == VARQ_PATH_SPLIT && lq > VARQ_SPLIT_MAX_LQ) return VARQ_ERR_UNSUPPORTED;
+  return VARQ_OK;
+}
+
+static void fill_dense(AttnArgs& a, int batch, int heads, int head_dim, int64_t n_tokens, int lq) {
+  std::memset(&a, 0, sizeof(a));
+  a.batch = batch;
+  a.heads = heads;
+  a.head_dim = head_dim;
+  a.lq = lq;
+  a.t_att = static_cast<int32_t>(n_tokens);
+}
+
+size_t varq_dense_attention_workspace(int batch, int heads, int head_dim, int lq, int64_t n_tokens, int path) {
+  if (check_dense(batch, heads, head_dim, n_tokens, lq, path) != VARQ_OK) return 0;
+  if (choose_path(lq, path) != VARQ_PATH_SPLIT) return 0;
+  AttnArgs a;
+  fill_dense(a, batch, heads, head_dim, n_tokens, lq);
+  return varq::split_kv_workspace_bytes(batch, heads, lq, head_dim, varq::dense_splits(a));
+}
+
+int varq_dense_attention(int batch, int heads, int head_dim, int64_t n_tokens, const void* q, int64_t q_sb,
+                         int64_t q_sh, int64_t q_st, int lq, const void* k, int64_t k_sb, int64_t k_sh, int64_t k_st,
+                         const void* v, int64_t v_sb, int64_t v_sh, int64_t v_st, float softmax_scale, void* out,
+                         int64_t o_sb, int64_t o_sh, int64_t o_st, float* lse, void* workspace,
+                         size_t workspace_bytes, int path, uint32_t* dev_status, void* stream) {
+  int rc = check_dense(batch, heads, head_dim, n_tokens, lq, path);
+  if (rc != VARQ_OK) return rc;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return VARQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VARQ_ERR_ALIGNMENT;
+  for (int64_t st : {q_sb, q_sh, q_st, k_sb, k_sh, k_st, v_sb, v_sh, v_st, o_sb, o_sh, o_st})
+    if (!stride_ok(st)) return VARQ_ERR_ALIGNMENT;
+  AttnArgs a;
+  fill_dense(a, batch, heads, head_dim, n_tokens, lq);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.q_sb = q_sb;
+  a.q_sh = q_sh;
+  a.q_st = q_st;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.o_sb = o_sb;
+  a.o_sh = o_sh;
+  a.o_st = o_st;
+  a.lse = lse;
+  a.dev_status = dev_status;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(float(head_dim));
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  if (choose_path(lq, path) == VARQ_PATH_SPLIT) {
+    a.kv_split = 1;
+    a.n_splits = varq::dense_splits(a);
+    const size_t need = varq::split_kv_workspace_bytes(batch, heads, lq, head_dim, a.n_splits);
+    if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
+    a.workspace = static_cast<float*>(workspace);
+  }
+  const varq::DenseTensor kt{k, k_sb, k_sh, k_st}, vt{v, v_sb, v_sh, v_st};
+  return varq::launch_attention_dense(a, kt, vt, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -20,6 +20,7 @@ __all__ = [
     "PATH_AUTO", "PATH_TENSOR", "PATH_SPLIT", "SPLIT_MAX_LQ",
     "DEV_NONFINITE", "DEV_META_OVERFLOW", "DEV_TIMEOUT",
     "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "varq_quantize_pack_launches",
+    "varq_dense_attention", "varq_dense_attention_workspace",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvarq.so")
@@ -85,6 +86,13 @@ def lib() -> ctypes.CDLL:
             _c_p, _c_p, _c_p, _c_p, _c_int, _c_f, _c_p, _c_p,
             _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_int, _c_p, _c_p]
         L.varq_packed_attention.restype = _c_int
+        L.varq_dense_attention_workspace.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_i64, _c_int]
+        L.varq_dense_attention_workspace.restype = _c_sz
+        L.varq_dense_attention.argtypes = [
+            _c_int, _c_int, _c_int, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_int,
+            _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_f,
+            _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_int, _c_p, _c_p]
+        L.varq_dense_attention.restype = _c_int
         L.varq_status_string.argtypes = [_c_int]
         L.varq_status_string.restype = ctypes.c_char_p
         L.varq_abi_version.argtypes = []
@@ -255,3 +263,32 @@ def varq_packed_attention_noalloc(layout: CacheLayout, q: torch.Tensor, k_packed
             _ptr(rope_cos), _ptr(rope_sin), _ptr(out), out.stride(0), out.stride(1), out.stride(2),
             _ptr(lse), _ptr(dev_status), _stream(stream))
     _check(rc, "varq_packed_attention_noalloc")
+
+
+def varq_dense_attention_workspace(batch: int, heads: int, head_dim: int, lq: int, n_tokens: int,
+                                   path: int = PATH_AUTO) -> int:
+    return int(lib().varq_dense_attention_workspace(batch, heads, head_dim, lq, n_tokens, path))
+
+
+def varq_dense_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                         softmax_scale: float = 0.0, lse: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO,
+                         dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Attention of ``q`` (bf16 ``[B, H, lq, D]``) over dense bf16 ``k, v``
+    (``[B, H, T, D]``): the attention half of the unfused baseline."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, n, torch.bfloat16)
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError(f"{n} must be [B, H, rows, D] with contiguous channels")
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    B, H, lq, D = q.shape
+    if k.shape != v.shape or k.shape[:2] != (B, H) or k.shape[3] != D:
+        raise ValueError("k and v must be [B, H, T, D] matching q")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().varq_dense_attention(
+        B, H, D, k.shape[2], _ptr(q), q.stride(0), q.stride(1), q.stride(2), lq,
+        _ptr(k), k.stride(0), k.stride(1), k.stride(2), _ptr(v), v.stride(0), v.stride(1), v.stride(2),
+        float(softmax_scale), _ptr(out), out.stride(0), out.stride(1), out.stride(2), _ptr(lse), _ptr(workspace),
+        ws_bytes, path, _ptr(dev_status), _stream(stream))
+    _check(rc, "varq_dense_attention")

@@ -157,6 +157,37 @@ def test_attention_errors():
     assert V.varq_packed_attention_workspace(L, 4, 3, V.PATH_TENSOR) == 0
 
 
+def test_dense_attention_errors():
+    lib = V.lib()
+    P = ctypes.c_void_p
+
+    def call(B=2, H=4, D=128, T=1000, lq=64, q=FAKE, k=FAKE, v=FAKE, out=FAKE, kst=128, scale=0.0, ws=None, wsb=0,
+             path=0):
+        return lib.varq_dense_attention(B, H, D, T, P(q) if q else None, 8, 8, 128, lq, P(k) if k else None, 8, 8,
+                                        kst, P(v) if v else None, 8, 8, 128, scale, P(out) if out else None, 8, 8,
+                                        128, None, P(ws) if ws else None, wsb, path, None, None)
+
+    assert call(B=0) == INVALID
+    assert call(lq=0) == INVALID
+    assert call(T=0) == INVALID
+    assert call(D=96) == UNSUPPORTED
+    assert call(q=None) == INVALID
+    assert call(k=None) == INVALID
+    assert call(out=None) == INVALID
+    assert call(path=5) == INVALID
+    assert call(scale=float("inf")) == INVALID
+    assert call(k=FAKE + 8) == ALIGN
+    assert call(kst=36) == ALIGN
+    assert call(lq=64, path=2) == UNSUPPORTED   # split path serves lq <= 16
+    assert call(lq=4) == WORKSPACE
+    need = V.varq_dense_attention_workspace(2, 4, 128, 4, 1000)
+    assert need > 0
+    assert call(lq=4, ws=FAKE, wsb=need - 4) == WORKSPACE
+    assert call(lq=4, ws=FAKE + 4, wsb=need) == ALIGN
+    assert V.varq_dense_attention_workspace(2, 4, 128, 200, 1000) == 0
+    assert V.varq_dense_attention_workspace(2, 4, 128, 4, 1000, V.PATH_TENSOR) == 0
+
+
 def test_status_strings():
     for c in (OK, INVALID, UNSUPPORTED, CUDA, WORKSPACE, ALIGN):
         assert V.varq_status_string(c).startswith("VARQ_")
