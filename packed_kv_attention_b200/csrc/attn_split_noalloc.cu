@@ -133,7 +133,9 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   rc = scratch_on_current_device(&scratch);
   if (rc != VARQ_OK) return rc;
   a.workspace = scratch;
-  const cudaError_t e = dec ? varq::launch_attention_decode(a, static_cast<cudaStream_t>(stream))
-                            : varq::launch_attention_tc(a, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = dec                              ? varq::launch_attention_decode(a, s)
+                        : varq::use_swap_ab_kernel(a) ? varq::launch_attention_swap_ab(a, s)
+                                                      : varq::launch_attention_tc(a, s);
   return e == cudaSuccess ? VARQ_OK : VARQ_ERR_CUDA;
 }

@@ -261,134 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp >= kDequantWarp0 || (NQ == 1 && warp >= 4)) {
     // ------------------------------------------------------------- dequant
     const int dt = warp >= kDequantWarp0 ? tid - kDequantWarp0 * 32 : kDequantThreads + tid - 128;
-    const int d = dt % D;
-    const int part = dt / D;
-    const int64_t bh = int64_t(b) * a.heads + h;
-    const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + d;
-    const uint32_t* mgv = a.v_meta + bh * a.n_blocks_total * D + d;
-    const int nblk = a.n_cached_blocks;
-    // (scale, min) words of this thread's channel for block blk and blk + 1,
-    // K and V, loaded one block ahead so a tile never waits on them
-    uint32_t mk_cur = __ldg(mgk), mv_cur = __ldg(mgv);
-    uint32_t mk_next = nblk > 1 ? __ldg(mgk + D) : 0u, mv_next = nblk > 1 ? __ldg(mgv + D) : 0u;
-    int blk = 0;  // block of the current tile's first token (monotone)
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % C::PST;
-      const int tok0 = (tile0 + j) * C::NKV;
-      while (tok0 >= sm_bs[blk + 1]) {
-        ++blk;
-        mk_cur = mk_next;
-        mv_cur = mv_next;
-        const bool more = blk + 1 < nblk;
-        mk_next = more ? __ldg(mgk + int64_t(blk + 1) * D) : 0u;
-        mv_next = more ? __ldg(mgv + int64_t(blk + 1) * D) : 0u;
-      }
-      const int blk_lo = blk;
-      if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
-      const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
-      bool ok = true;
-      for (int tensor = 0; tensor < 2 && ok; ++tensor) {
-        const int nbuf = tensor == 0 ? C::KST : C::VST;
-        const int buf = j % nbuf;
-        uint64_t* freeb = tensor == 0 ? &bars->kfree[buf] : &bars->vfree[buf];
-        if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint32_t* words = reinterpret_cast<const uint32_t*>(sb + tensor * C::WORDS_BYTES);
-        uint8_t* dst = smem + (tensor == 0 ? C::OFF_K : C::OFF_V) + buf * C::KV_BYTES + d * 128;
-        int cb = blk_lo;         // current block
-        int nb = sm_bs[cb + 1];  // its end
-        const uint32_t m_cur = tensor == 0 ? mk_cur : mv_cur;
-        const uint32_t m_next = tensor == 0 ? mk_next : mv_next;
-        const uint32_t* m_glob = tensor == 0 ? mgk : mgv;
-        const float msc = (ROPE && tensor == 0) ? exp2i(kexp) : 1.0f;  // exact: commutes with every rounding below
-        auto meta_of = [&](int k) -> float2 {
-          const uint32_t w = k == blk_lo ? m_cur : (k == blk_lo + 1 ? m_next : __ldg(m_glob + int64_t(k) * D));
-          const float2 sm0 = meta_unpack(w);
-          return make_float2(sm0.x * msc, sm0.y * msc);
-        };
-        float2 sm = meta_of(cb);
-        // exact code -> value without a shift per code: the code at bit r of
-        // a shifted word becomes 2^23 + q 2^r (OR into the mantissa of 2^23),
-        // then fma(., s 2^-r, -2^(23-r) s) = q s exactly and + m rounds once,
-        // which is fmaf(q, s, m).
-        float cs[C::CPC], cc[C::CPC];
-        auto set_consts = [&](float s) {
-#pragma unroll
-          for (int rr = 0; rr < C::CPC; ++rr) {
-            cs[rr] = s * __uint_as_float(uint32_t(127 - rr * BITS) << 23);
-            cc[rr] = -s * __uint_as_float(uint32_t(127 + 23 - rr * BITS) << 23);
-          }
-        };
-        set_consts(sm.x);
-        for (int g = part; g < C::NG; g += C::TPC) {
-          const int tg = tok0 + g * C::GT;
-          uint32_t wv[C::GW];
-#pragma unroll
-          for (int i = 0; i < C::GW; ++i) wv[i] = words[(g * C::GW + i) * D + d];
-          float x[C::GT];
-          if (tg + C::GT <= nb && tg + C::GT <= t_att) {
-#pragma unroll
-            for (int jt = 0; jt < C::GT; ++jt) {
-              const int jj = jt % CPW;
-              const int chunk = jj / C::CPC, rr = jj % C::CPC;
-              const uint32_t ws = wv[jt / CPW] >> (chunk * C::CPC * BITS);
-              const float f = __uint_as_float((ws & (MASK << (rr * BITS))) | 0x4B000000u);
-              x[jt] = __fadd_rn(__fmaf_rn(f, cs[rr], cc[rr]), sm.y);
-            }
-          } else {
-#pragma unroll
-            for (int jt = 0; jt < C::GT; ++jt) {
-              const int t = tg + jt;
-              float v = 0.0f;
-              if (t < t_att) {
-                if (t >= nb) {
-                  while (t >= sm_bs[cb + 1]) ++cb;
-                  nb = sm_bs[cb + 1];
-                  sm = meta_of(cb);
-                  set_consts(sm.x);
-                }
-                const uint32_t q = (wv[jt / CPW] >> ((jt % CPW) * BITS)) & MASK;
-                v = __fmaf_rn(small_uint_to_float(q), sm.x, sm.y);
-              }
-              x[jt] = v;
-            }
-          }
-          if (ROPE && tensor == 0) {
-            // pre-RoPE key mode: rotate pair (2i, 2i+1) of every token after
-            // dequantization; the partner channel lives in the neighbour lane
-#pragma unroll
-            for (int jt = 0; jt < C::GT; ++jt) {
-              const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
-              const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
-              const int t = tg + jt;
-              float c = 1.0f, s = 0.0f;
-              if (t < t_att) {
-                c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
-                s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
-              }
-              x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
-            }
-          }
-#pragma unroll
-          for (int c = 0; c < C::GC; ++c) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              pk[k] = (QK_F16 && tensor == 0) ? pack_f16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1])
-                                              : pack_bf16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1]);
-            const int tt = g * C::GT + c * 8;  // token within the tile
-            const uint32_t off = (tt >> 6) * (D * 128) + ((((tt >> 3) & 7) ^ (d & 7)) << 4);
-            *reinterpret_cast<uint4*>(dst + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-        fence_async_smem();
-        mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
-      }
-      if (!ok || *abort_flag) break;
-      mbar_arrive(&bars->empty[st]);
-    }
+    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, dt, b, h, tile0, ntiles, kexp);
   } else if ((warp >> 2) < NQ) {
     // ------------------------------------------------------------- softmax
     const int i = warp >> 2, r = (warp & 3) * 32 + lane;

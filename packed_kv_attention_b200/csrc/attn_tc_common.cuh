@@ -37,7 +37,9 @@ struct Barriers {
   uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
-  uint32_t kmax[20];              // pre-RoPE keys: per-warp largest |min| + (2^b - 1) scale
+  uint32_t kmax[24];              // pre-RoPE keys: per-warp largest |min| + (2^b - 1) scale
+  alignas(16) uint32_t flag[2][4];  // swap-AB split kernel: per-warp softmax votes, by tile parity
+  uint64_t sync[2], sync2[2];     // swap-AB split kernel: softmax-warp exchanges, by tile parity
 };
 static_assert(sizeof(Barriers) <= 512, "the barriers sit below the block-start table");
 
@@ -377,6 +379,171 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
     }
     if (row < a.lq && a.lse != nullptr)
       a.lse[(int64_t(b) * a.heads + h) * a.lq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+  }
+}
+
+
+// The dequant warps of the single-CTA tensor-core kernels.  Thread dt owns
+// channel d = dt % D and the dequant groups part, part + TPC, ... of every KV
+// tile (a group = GT tokens = whole packed words and whole 16-byte chunks).
+// Per tile: wait for the packed stage, then for each of K and V wait until
+// the previous MMAs have released the 16-bit tile buffer, unpack and
+// dequantize the channel's codes to x_hat = bf16(fmaf(q, s, min)) and write
+// them straight into the 128-byte-swizzled operand layout
+//   [NKV/64 panels][D rows (channels)][64 tokens]
+// (MN-major B of S = Q K^T, K-major B of O = P V; in the swap-AB split kernel
+// the MN-major A of S^T = K Q^T and the K-major A of O^T = V^T P^T).  Pre-RoPE
+// keys are rotated pair-wise after dequantization (partner channel in the
+// neighbour lane) and rounded to fp16, scaled by 2^kexp (exact).  The
+// per-block (scale, min) words of the channel for the current and the next
+// block are held in registers.
+//
+// C provides CPW, GT, GW, GC, CPC, NKV, NG, TPC, PST, KST, VST, OFF_STAGE,
+// STAGE_BYTES, WORDS_BYTES, OFF_K, OFF_V, KV_BYTES and DEQ (the number of
+// dequant threads, the arrival count of kready/vready/empty).
+template <class C, int BITS, int D, bool ROPE>
+__device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, uint8_t* smem, const int* sm_bs, int dt,
+                                             int b, int h, int tile0, int ntiles, int kexp) {
+  constexpr int CPW = C::CPW;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr bool QK_F16 = ROPE;
+  volatile int* abort_flag = &bars->abort_flag;
+  const int t_att = a.t_att;
+  const int d = dt % D;
+  const int part = dt / D;
+  const int64_t bh = int64_t(b) * a.heads + h;
+  const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + d;
+  const uint32_t* mgv = a.v_meta + bh * a.n_blocks_total * D + d;
+  const int nblk = a.n_cached_blocks;
+  // (scale, min) words of this thread's channel for block blk and blk + 1,
+  // K and V, loaded one block ahead so a tile never waits on them
+  uint32_t mk_cur = __ldg(mgk), mv_cur = __ldg(mgv);
+  uint32_t mk_next = nblk > 1 ? __ldg(mgk + D) : 0u, mv_next = nblk > 1 ? __ldg(mgv + D) : 0u;
+  int blk = 0;  // block of the current tile's first token (monotone)
+  for (int j = 0; j < ntiles; ++j) {
+    const int st = j % C::PST;
+    const int tok0 = (tile0 + j) * C::NKV;
+    while (tok0 >= sm_bs[blk + 1]) {
+      ++blk;
+      mk_cur = mk_next;
+      mv_cur = mv_next;
+      const bool more = blk + 1 < nblk;
+      mk_next = more ? __ldg(mgk + int64_t(blk + 1) * D) : 0u;
+      mv_next = more ? __ldg(mgv + int64_t(blk + 1) * D) : 0u;
+    }
+    const int blk_lo = blk;
+    if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
+    const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
+    bool ok = true;
+    for (int tensor = 0; tensor < 2 && ok; ++tensor) {
+      const int nbuf = tensor == 0 ? C::KST : C::VST;
+      const int buf = j % nbuf;
+      uint64_t* freeb = tensor == 0 ? &bars->kfree[buf] : &bars->vfree[buf];
+      if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t* words = reinterpret_cast<const uint32_t*>(sb + tensor * C::WORDS_BYTES);
+      uint8_t* dst = smem + (tensor == 0 ? C::OFF_K : C::OFF_V) + buf * C::KV_BYTES + d * 128;
+      int cb = blk_lo;         // current block
+      int nb = sm_bs[cb + 1];  // its end
+      const uint32_t m_cur = tensor == 0 ? mk_cur : mv_cur;
+      const uint32_t m_next = tensor == 0 ? mk_next : mv_next;
+      const uint32_t* m_glob = tensor == 0 ? mgk : mgv;
+      const float msc = (ROPE && tensor == 0) ? exp2i(kexp) : 1.0f;  // exact: commutes with every rounding below
+      auto meta_of = [&](int k) -> float2 {
+        const uint32_t w = k == blk_lo ? m_cur : (k == blk_lo + 1 ? m_next : __ldg(m_glob + int64_t(k) * D));
+        const float2 sm0 = meta_unpack(w);
+        return make_float2(sm0.x * msc, sm0.y * msc);
+      };
+      float2 sm = meta_of(cb);
+      // exact code -> value without a shift per code: the code at bit r of a
+      // shifted word becomes 2^23 + q 2^r (OR into the mantissa of 2^23), then
+      // fma(., s 2^-r, -2^(23-r) s) = q s exactly and + m rounds once, which
+      // is fmaf(q, s, m).  Two codes per packed fp32x2 fma and add (the same
+      // IEEE roundings per half).
+      float cs[C::CPC], cc[C::CPC];
+      auto set_consts = [&](float s) {
+#pragma unroll
+        for (int rr = 0; rr < C::CPC; ++rr) {
+          cs[rr] = s * __uint_as_float(uint32_t(127 - rr * BITS) << 23);
+          cc[rr] = -s * __uint_as_float(uint32_t(127 + 23 - rr * BITS) << 23);
+        }
+      };
+      set_consts(sm.x);
+      for (int g = part; g < C::NG; g += C::TPC) {
+        const int tg = tok0 + g * C::GT;
+        uint32_t wv[C::GW];
+#pragma unroll
+        for (int i = 0; i < C::GW; ++i) wv[i] = words[(g * C::GW + i) * D + d];
+        float x[C::GT];
+        if (tg + C::GT <= nb && tg + C::GT <= t_att) {
+          auto code_f = [&](int jt) {
+            const int jj = jt % CPW;
+            const int chunk = jj / C::CPC, rr = jj % C::CPC;
+            const uint32_t ws = wv[jt / CPW] >> (chunk * C::CPC * BITS);
+            return __uint_as_float((ws & (MASK << (rr * BITS))) | 0x4B000000u);
+          };
+          const uint64_t m2 = f2_pack(sm.y, sm.y);
+#pragma unroll
+          for (int jt = 0; jt < C::GT; jt += 2) {
+            const int r0 = (jt % CPW) % C::CPC, r1 = ((jt + 1) % CPW) % C::CPC;
+            const uint64_t y = f2_add(f2_fma(f2_pack(code_f(jt), code_f(jt + 1)), f2_pack(cs[r0], cs[r1]),
+                                             f2_pack(cc[r0], cc[r1])),
+                                      m2);
+            f2_unpack(y, x[jt], x[jt + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int jt = 0; jt < C::GT; ++jt) {
+            const int t = tg + jt;
+            float v = 0.0f;
+            if (t < t_att) {
+              if (t >= nb) {
+                while (t >= sm_bs[cb + 1]) ++cb;
+                nb = sm_bs[cb + 1];
+                sm = meta_of(cb);
+                set_consts(sm.x);
+              }
+              const uint32_t q = (wv[jt / CPW] >> ((jt % CPW) * BITS)) & MASK;
+              v = __fmaf_rn(small_uint_to_float(q), sm.x, sm.y);
+            }
+            x[jt] = v;
+          }
+        }
+        if (ROPE && tensor == 0) {
+          // pre-RoPE key mode: rotate pair (2i, 2i+1) of every token after
+          // dequantization; the partner channel lives in the neighbour lane
+#pragma unroll
+          for (int jt = 0; jt < C::GT; ++jt) {
+            const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
+            const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
+            const int t = tg + jt;
+            float c = 1.0f, s = 0.0f;
+            if (t < t_att) {
+              c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
+              s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
+            }
+            x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < C::GC; ++c) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            pk[k] = (QK_F16 && tensor == 0) ? pack_f16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1])
+                                            : pack_bf16x2(x[c * 8 + 2 * k], x[c * 8 + 2 * k + 1]);
+          const int tt = g * C::GT + c * 8;  // token within the tile
+          const uint32_t off = (tt >> 6) * (D * 128) + ((((tt >> 3) & 7) ^ (d & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
+    }
+    if (!ok || *abort_flag) break;
+    mbar_arrive(&bars->empty[st]);
   }
 }
 

@@ -126,6 +126,11 @@ constexpr int kDecodeMaxLq = 2;
 bool use_decode_kernel(const AttnArgs& a);
 int split_kv_decode_splits(const AttnArgs& a);
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);
+// Split-KV form for lq <= 16 and head_dim 128 with the operands swapped
+// (S^T = K Q^T: cached tokens on the 128-row MMA side), writing the same
+// partials and running the same merge.
+bool use_swap_ab_kernel(const AttnArgs& a);
+cudaError_t launch_attention_swap_ab(const AttnArgs& a, cudaStream_t stream);
 // Attention over dense bf16 K and V (the unfused baseline's second half), on
 // the tensor cores with TMA-loaded tiles; with kv_split, the split-KV form plus
 // the combine.  Returns a varq_status (VARQ_ERR_UNSUPPORTED when a tensor map

@@ -224,7 +224,9 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
   a.workspace = static_cast<float*>(workspace);
-  return launch_status(dec ? varq::launch_attention_decode(a, s) : varq::launch_attention_tc(a, s));
+  if (dec) return launch_status(varq::launch_attention_decode(a, s));
+  return launch_status(varq::use_swap_ab_kernel(a) ? varq::launch_attention_swap_ab(a, s)
+                                                   : varq::launch_attention_tc(a, s));
 }
 
 static int check_dense(int batch, int heads, int head_dim, int64_t n_tokens, int lq, int path) {
