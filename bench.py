@@ -173,6 +173,8 @@ class Pipeline:
         # quantize+pack of K and V plus the attention (split-KV: split + combine)
         self.launches_per_step = 2 * V.varq_quantize_pack_launches(self.L) + (1 if ws == 0 else 2)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        # made on the default stream; the library's launches go to another one
+        torch.cuda.synchronize(device)
 
     def step(self, stream, ev=None):
         V = self.V
@@ -321,6 +323,7 @@ def run_reference(args, w, rank, world):
 def _event_times(fn, stream, iters):
     """Per-iteration device times (ms) of fn() on stream, each bracketed by
     CUDA events (every input below exceeds the 126 MB L2)."""
+    torch.cuda.synchronize()
     times = []
     for _ in range(iters):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -357,6 +360,7 @@ def measure_rows(dev, stream, peaks, iters=5):
     for bits in (2, 3, 4, 8):
         L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, bs)
         kp, km = V.alloc_cache(L, dev)
+        torch.cuda.synchronize()  # made on the default stream, used on `stream`
         for _ in range(3):
             V.varq_quantize_pack(L, k, kp, km, dev_status=st, stream=stream)
         tq = statistics.median(_event_times(
@@ -375,6 +379,7 @@ def measure_rows(dev, stream, peaks, iters=5):
 
     # a9: split-KV attention over the INT4 sweep cache (K and V share the packed words here)
     vp4, vm4 = V.alloc_cache(L4, dev)
+    torch.cuda.synchronize()
     V.varq_quantize_pack(L4, v, vp4, vm4, dev_status=st, stream=stream)
     split = {}
     for lq in (1, 4, 16):
@@ -386,6 +391,7 @@ def measure_rows(dev, stream, peaks, iters=5):
         def run():
             V.varq_packed_attention(L4, q, kp4, km4, vp4, vm4, o, workspace=ws, path=V.PATH_SPLIT,
                                     dev_status=st, stream=stream)
+        torch.cuda.synchronize()
         for _ in range(3):
             run()
         t = statistics.median(_event_times(run, stream, iters))
@@ -400,6 +406,7 @@ def measure_rows(dev, stream, peaks, iters=5):
     # a8: pre-RoPE keys on the tensor path (Self-Forcing-like layer)
     w = synth.WORKLOADS["self_forcing"]
     pipe = Pipeline(w, 4, w.lq[-1], dev, seed=4)
+    torch.cuda.synchronize()
     pipe.step(stream)
     torch.cuda.synchronize()
 
@@ -407,6 +414,7 @@ def measure_rows(dev, stream, peaks, iters=5):
         V.varq_packed_attention(pipe.L, pipe.q, pipe.kp, pipe.km, pipe.vp, pipe.vm, pipe.out,
                                 rope_cos=pipe.cos, rope_sin=pipe.sin, workspace=pipe.ws,
                                 dev_status=st, stream=stream)
+    torch.cuda.synchronize()
     for _ in range(2):
         attn()
     t = statistics.median(_event_times(attn, stream, 3))
@@ -512,6 +520,9 @@ def measure_rows(dev, stream, peaks, iters=5):
 
 
 def _median_ms(fn, stream, iters, warm=2):
+    # the inputs and buffers were made on the default stream, the library runs
+    # on `stream`: finish the former before the first launch
+    torch.cuda.synchronize()
     for _ in range(warm):
         fn()
     return statistics.median(_event_times(fn, stream, iters))
@@ -538,6 +549,7 @@ def measure_fused_vs_unfused(dev, stream, peaks, bits=4, iters=3):
     kp, km = V.alloc_cache(L, dev)
     vp, vm = V.alloc_cache(L, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()  # inputs and buffers come from the default stream
     V.varq_quantize_pack(L, data["k"], kp, km, dev_status=st, stream=stream)
     V.varq_quantize_pack(L, data["v"], vp, vm, dev_status=st, stream=stream)
     kd, vd = data["k"], data["v"]  # reused as the dense workspaces (overwritten by unpack+dequant)

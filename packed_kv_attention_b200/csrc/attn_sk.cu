@@ -29,6 +29,10 @@
 // positions; they are summed over the 128 threads once at the end.  The
 // warps exchange votes and maxima through shared memory, synchronised by
 // mbarriers with bounded waits, so a warp that aborts never blocks the others.
+// Every exchange barrier's phases follow the number of times it has been used
+// (the vote barrier once per tile, the maximum barrier once per rescale): a
+// wait that named a phase by the tile index could be one phase off and return
+// before the other warps had arrived.
 // The CTA writes its unnormalised partial (O, m in the log2 domain, l) per
 // query row; attn_combine.cu merges the ranges.
 #include <algorithm>
@@ -262,6 +266,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     // [2 panels of 64 tokens][16 rows][128 B], 128-byte swizzle
     const uint32_t p_thread = uint32_t(t >> 6) * (kSkN * 128) + uint32_t(t & 7) * 2;
     const uint32_t p_chunk = uint32_t((t & 63) >> 3);
+    // rescale exchanges so far: the second exchange barrier is used only on
+    // tiles that rescale, so its phases follow this count, not the tile index
+    int n_resc = 0;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       ok = wait_all(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag);
@@ -298,8 +305,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
           const uint32_t u = __reduce_max_sync(0xFFFFFFFFu, f2ord(y[i]));
           if (lane == i) sm_tmax[warp * kSkN + i] = u;
         }
-        mbar_arrive(&bars->sync2[j & 1]);
-        ok = wait_all(&bars->sync2[j & 1], (j >> 1) & 1, abort_flag);
+        mbar_arrive(&bars->sync2[n_resc & 1]);
+        ok = wait_all(&bars->sync2[n_resc & 1], (n_resc >> 1) & 1, abort_flag);
+        ++n_resc;
         if (!ok) break;
         // O^T holds the earlier tiles once P V(j - 1) has finished (P V(j - 2)
         // is waited for again below, every tile: it has long completed)
