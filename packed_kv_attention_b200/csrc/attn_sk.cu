@@ -78,17 +78,21 @@ struct SkCfg {
   static constexpr uint32_t need(int pst, int kst, int vst) {
     return Q_BYTES + 2 * P_BYTES + (kst + vst) * KV_BYTES + pst * STAGE_BYTES + TMAX_BYTES + kBarBytes;
   }
+  // buffer counts (packed stages, K tiles, V tiles): the deepest packed-stage
+  // prefetch first (a copy is issued PST - 1 tiles ahead of its use, which
+  // must cover the HBM latency at this kernel's per-tile rate), then double
+  // buffered K and V tiles
+  static constexpr int OPTS[7][3] = {{4, 2, 2}, {3, 2, 2}, {2, 2, 2}, {2, 2, 1}, {1, 2, 2}, {2, 1, 1}, {1, 1, 1}};
   static constexpr int pick() {
-    const int opts[5][3] = {{2, 2, 2}, {2, 2, 1}, {1, 2, 2}, {2, 1, 1}, {1, 1, 1}};
-    for (int o = 0; o < 5; ++o)
-      if (need(opts[o][0], opts[o][1], opts[o][2]) <= kSmemUsable) return o;
+    for (int o = 0; o < 7; ++o)
+      if (need(OPTS[o][0], OPTS[o][1], OPTS[o][2]) <= kSmemUsable) return o;
     return -1;
   }
   static constexpr int OPT = pick();
   static_assert(OPT >= 0, "shared memory budget");
-  static constexpr int PST = (OPT == 2 || OPT == 4) ? 1 : 2;
-  static constexpr int KST = (OPT == 3 || OPT == 4) ? 1 : 2;
-  static constexpr int VST = (OPT == 0 || OPT == 2) ? 2 : 1;
+  static constexpr int PST = OPTS[OPT][0];
+  static constexpr int KST = OPTS[OPT][1];
+  static constexpr int VST = OPTS[OPT][2];
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_P = OFF_Q + Q_BYTES;
   static constexpr uint32_t OFF_K = OFF_P + 2 * P_BYTES;
@@ -143,9 +147,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
 
   // ------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::PST; ++i) {
       mbar_init(&bars->full[i], 1);
       mbar_init(&bars->empty[i], C::DEQ);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->kready[i], C::DEQ);
       mbar_init(&bars->kfree[i], 1);
       mbar_init(&bars->vready[i], C::DEQ);

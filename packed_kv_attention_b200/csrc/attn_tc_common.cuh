@@ -27,7 +27,7 @@ template <int NQ>
 __host__ __device__ constexpr uint32_t col_o(int i) { return uint32_t(NQ) * 128u + uint32_t(i) * 128u; }
 
 struct Barriers {
-  uint64_t full[2], empty[2];     // packed stage filled by TMA / released by dequant
+  uint64_t full[4], empty[4];     // packed stage filled by TMA / released by dequant (up to 4 stages)
   uint64_t kready[3], kfree[3];   // 16-bit K tile written / consumed by all S MMAs (per K stage)
   uint64_t vready[3], vfree[3];   // 16-bit V tile written / consumed by all PV MMAs (per V stage)
   // indexed by query tile i, or by KV tile & 1 where S is double-buffered
