@@ -428,12 +428,25 @@ def measure_rows(dev, stream, peaks, iters=5):
     for _ in range(2):
         attn_post()
     t_post = statistics.median(_event_times(attn_post, stream, 3))
+
+    # the same pre-RoPE layer with the angles computed in the kernel from the
+    # (frame, row, column) schedule the tables describe
+    rope3d = V.Rope3d.make(1560, 52, synth.rope_axis_pairs(w.head_dim))
+
+    def attn_sched():
+        V.varq_packed_attention_rope3d(pipe.L, pipe.q, pipe.kp, pipe.km, pipe.vp, pipe.vm, pipe.out, rope3d,
+                                       workspace=pipe.ws, dev_status=st, stream=stream)
+    for _ in range(2):
+        attn_sched()
+    t_sched = statistics.median(_event_times(attn_sched, stream, 3))
     rows["a8_pre_rope_attention"] = {
         "workload": f"self_forcing: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} Lq={w.lq[-1]} INT4 pre-RoPE",
         "bound": "tensor", "ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12,
         "frac_tensor": fl / (t * 1e-3) / 1e12 / tflops_peak,
         "frac_tensor_sustained": fl / (t * 1e-3) / 1e12 / tflops_sus,
-        "post_rope_ms": t_post, "post_rope_TFLOP/s": fl / (t_post * 1e-3) / 1e12}
+        "post_rope_ms": t_post, "post_rope_TFLOP/s": fl / (t_post * 1e-3) / 1e12,
+        "schedule_ms": t_sched, "schedule_TFLOP/s": fl / (t_sched * 1e-3) / 1e12,
+        "schedule_frac_tensor": fl / (t_sched * 1e-3) / 1e12 / tflops_peak}
     del pipe
     torch.cuda.empty_cache()
 
@@ -617,6 +630,8 @@ def measure_longlive(dev, stream, peaks, iters=3):
     data = synth.make_inputs(w, lq=w.lq[-1], seed=7, device=dev)
     bs = data["block_start"]
     cos, sin = data["rope_cos"], data["rope_sin"]
+    rope3d = V.Rope3d.make(1560, 52, synth.rope_axis_pairs(w.head_dim))
+    tables = 2 * cos.numel() * cos.element_size()
     lq = w.lq[-1]
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     o = torch.empty_like(data["q"])
@@ -633,8 +648,12 @@ def measure_longlive(dev, stream, peaks, iters=3):
         def attn():
             V.varq_packed_attention(L, data["q"], kp, km, vp, vm, o, rope_cos=cos, rope_sin=sin, dev_status=st,
                                     stream=stream)
+
+        def attn_sched():
+            V.varq_packed_attention_rope3d(L, data["q"], kp, km, vp, vm, o, rope3d, dev_status=st, stream=stream)
         t_q = _median_ms(quant, stream, iters)
         t_a = _median_ms(attn, stream, iters)
+        t_s = _median_ms(attn_sched, stream, iters)
         fl = attention_flops(w, lq)
         qb = quant_bytes(L, w)
         ab = attention_bytes(L, w, lq, True)
@@ -643,10 +662,13 @@ def measure_longlive(dev, stream, peaks, iters=3):
                              "quant_pack_frac_hbm": qb / (t_q * 1e-3) / 1e9 / peaks["hbm_gbs"],
                              "attention_ms": t_a, "attention_TFLOP/s": fl / (t_a * 1e-3) / 1e12,
                              "attention_bound": bound, "attention_frac": fr_a,
-                             "attention_frac_sustained": fl / (t_a * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+                             "attention_frac_sustained": fl / (t_a * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                             "schedule_attention_ms": t_s, "schedule_attention_TFLOP/s": fl / (t_s * 1e-3) / 1e12,
+                             "schedule_attention_frac": roofline_frac(fl, ab - tables, t_s, peaks)[0]}
         del kp, km, vp, vm
     res = {"workload": f"longlive: B={w.batch} H={w.heads} D={w.head_dim} T={w.n_tokens} blocks={w.n_blocks} "
-                       f"Lq={lq} pre-RoPE keys (3D RoPE tables)", **res, "device_status": int(st.item())}
+                       f"Lq={lq} pre-RoPE keys (3D RoPE tables; schedule_* = angles from the 1560-token "
+                       f"frame schedule in the kernel)", **res, "device_status": int(st.item())}
     del data, o
     torch.cuda.empty_cache()
     return res

@@ -229,6 +229,45 @@ VARQ_API int varq_packed_attention(const varq_cache_layout* layout,
                           int path, uint32_t* dev_status, void* stream);
 
 /*
+ * Rotary schedule of the 3D (frame, row, column) RoPE of video models, for
+ * varq_packed_attention_rope3d.  Token t lies in frame t / frame_tokens, at
+ * row (t % frame_tokens) / grid_w and column t % grid_w.  Key pair i belongs
+ * to the frame axis (i < pairs[0]), the row axis (i < pairs[0] + pairs[1]) or
+ * the column axis, as pair j of that axis's n = pairs[axis], and turns by
+ * position * base^(-j / n) radians.
+ */
+typedef struct varq_rope3d {
+  int32_t frame_tokens;     /* tokens per latent frame, a multiple of grid_w  */
+  int32_t grid_w;           /* tokens per latent row                          */
+  int32_t pairs[3];         /* rotary pairs of the frame, row, column axes;   */
+                            /* their sum is head_dim / 2                      */
+  float base;               /* > 0, e.g. 10000                                */
+} varq_rope3d;
+
+/*
+ * varq_packed_attention_rope3d -- varq_packed_attention in the pre-RoPE key
+ * mode with the rotation angles computed from token positions instead of read
+ * from [T, D/2] tables ([PAGE] "The block axis", Eq. 3: RoPE rotates each
+ * (2i, 2i+1) key pair; Appendix F: keys quantized before RoPE).  Every other
+ * argument as varq_packed_attention (whose rope_cos / rope_sin this replaces).
+ * Each CTA tabulates cos and sin of the angles its tokens use (the frames of
+ * its part of the cache, every row, every column) in shared memory,
+ * computed in double precision and rounded to fp32 -- the values a host
+ * table built the same way holds.  Returns VARQ_ERR_INVALID_ARG for a
+ * malformed schedule and VARQ_ERR_UNSUPPORTED when a CTA's table would not
+ * fit in shared memory beside the kernel's buffers (very many frames per
+ * CTA; the table path of varq_packed_attention has no such limit).
+ */
+VARQ_API int varq_packed_attention_rope3d(const varq_cache_layout* layout,
+                                          const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st, int lq,
+                                          const uint32_t* k_packed, const uint32_t* k_meta,
+                                          const uint32_t* v_packed, const uint32_t* v_meta,
+                                          int n_cached_blocks, float softmax_scale, const varq_rope3d* rope,
+                                          void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          int path, uint32_t* dev_status, void* stream);
+
+/*
  * varq_packed_attention_noalloc -- the split-KV attention of
  * varq_packed_attention (VARQ_PATH_SPLIT, lq <= VARQ_SPLIT_MAX_LQ) for
  * callers that cannot allocate device memory: a process whose allocator has

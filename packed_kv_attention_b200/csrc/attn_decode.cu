@@ -447,7 +447,7 @@ cudaError_t launch_dec_bits(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool use_decode_kernel(const AttnArgs& a) {
-  return a.kv_split && a.rope_cos == nullptr && a.lq <= kDecodeMaxLq;
+  return a.kv_split && !has_rope(a) && a.lq <= kDecodeMaxLq;
 }
 
 // About six CTAs per SM over the grid, each warp at least four steps long;

@@ -174,6 +174,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
   if constexpr (ROPE)
     rope_key_bound_partial<BITS, D, kSkThreads>(a.k_meta + (int64_t(b) * a.heads + h) * a.n_blocks_total * D,
                                                 a.n_cached_blocks, bars);
+  // rotary mode 2: the CTA's table of the 3D schedule, after the barrier region
+  float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
+  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * NKV) / a.rope_frame : 0;
+  if constexpr (ROPE)
+    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kSkThreads);
   // the 16-row query tile -> K-major swizzled smem (rows past lq are zero);
   // a row's 16 chunks are lanes 0-15 or 16-31 of one warp
   {
@@ -256,7 +261,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     }
   } else if (warp >= kSkDeqWarp0) {
     // ------------------------------------------------------------- dequant
-    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, tid - kSkDeqWarp0 * 32, b, h, tile0, ntiles, kexp);
+    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, tid - kSkDeqWarp0 * 32, b, h, tile0, ntiles, kexp, rope_tab,
+                                   rope_f0);
   } else {
     // ------------------------------------------------------------- softmax
     const int t = tid;                                   // TMEM lane: token t of S^T, channel t of O^T
@@ -423,10 +429,12 @@ template <int BITS, bool ROPE>
 cudaError_t launch_sk(const AttnArgs& a, cudaStream_t stream) {
   using C = SkCfg<BITS, 128>;
   auto kern = attn_sk_kernel<BITS, ROPE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  const uint32_t smem = C::SMEM + (ROPE ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
+  if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(unsigned(a.n_splits), unsigned(a.heads), unsigned(a.batch));
-  kern<<<grid, kSkThreads, C::SMEM, stream>>>(a);
+  kern<<<grid, kSkThreads, smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention_combine(a, stream);
@@ -434,7 +442,7 @@ cudaError_t launch_sk(const AttnArgs& a, cudaStream_t stream) {
 
 template <int BITS>
 cudaError_t launch_sk_bits(const AttnArgs& a, cudaStream_t s) {
-  return a.rope_cos != nullptr ? launch_sk<BITS, true>(a, s) : launch_sk<BITS, false>(a, s);
+  return has_rope(a) ? launch_sk<BITS, true>(a, s) : launch_sk<BITS, false>(a, s);
 }
 
 }  // namespace

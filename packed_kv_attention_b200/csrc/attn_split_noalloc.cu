@@ -106,6 +106,7 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
   a.v_meta = v_meta;
   a.rope_cos = rope_cos;
   a.rope_sin = rope_sin;
+  a.rope_mode = rope_cos != nullptr ? 1 : 0;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.o_sb = o_sb;
   a.o_sh = o_sh;

@@ -168,6 +168,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if constexpr (ROPE)
     rope_key_bound_partial<BITS, D, kThreads>(a.k_meta + (int64_t(b) * a.heads + h) * a.n_blocks_total * D,
                                               a.n_cached_blocks, bars);
+  // rotary mode 2: the CTA's table of the 3D schedule, after the barrier region
+  float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
+  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * C::NKV) / a.rope_frame : 0;
+  if constexpr (ROPE)
+    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kThreads);
   // query tiles -> K-major swizzled smem (rows past lq are zero).  The CH
   // chunks of a row are consecutive lanes of one warp in one pass, so with
   // fp16 operands they agree on the row's exponent by shuffles.
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp >= kDequantWarp0 || (NQ == 1 && warp >= 4)) {
     // ------------------------------------------------------------- dequant
     const int dt = warp >= kDequantWarp0 ? tid - kDequantWarp0 * 32 : kDequantThreads + tid - 128;
-    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, dt, b, h, tile0, ntiles, kexp);
+    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, dt, b, h, tile0, ntiles, kexp, rope_tab, rope_f0);
   } else if ((warp >> 2) < NQ) {
     // ------------------------------------------------------------- softmax
     const int i = warp >> 2, r = (warp & 3) * 32 + lane;
@@ -293,8 +298,11 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<BITS, D, NQ>;
   auto kern = attn_tc_kernel<BITS, D, NQ, ROPE>;
   // every CTA allocates all 512 TMEM columns: ask for enough shared memory
-  // that no second CTA is placed on the SM to wait for them
-  const uint32_t smem = std::max<uint32_t>(C::SMEM, kSmemUsable / 2 + 1024);
+  // that no second CTA is placed on the SM to wait for them (plus the rotary
+  // table of rope mode 2, which must fit)
+  const uint32_t extra = ROPE ? rope_table_bytes(a) : 0u;
+  if (C::SMEM + extra > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
+  const uint32_t smem = std::max<uint32_t>(C::SMEM + extra, kSmemUsable / 2 + 1024);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned((a.lq + NQ * BM - 1) / (NQ * BM) * (a.kv_split ? a.n_splits : 1)), a.heads, a.batch);
@@ -311,24 +319,18 @@ bool two_tiles(const AttnArgs& a) {
   return !a.kv_split && a.lq > BM && ctas >= 2 * 148;
 }
 
-// Tokens per KV tile for a bit width (Cfg<BITS, D, NQ>::NKV).
-int tile_tokens(int bits) {
-  const int cpw = 32 / bits;
-  int g = cpw, h = 16;
-  while (h != 0) {
-    const int t = g % h;
-    g = h;
-    h = t;
-  }
-  const int unit = cpw / g * 16;
-  return (128 / unit) * unit;
-}
-
+// Pre-RoPE keys reach this kernel only in the split-KV form (one query tile)
+// with 64 channels: the paired-CTA kernel takes the tensor path and the
+// swap-AB kernel the 128-channel split form.
 template <int BITS, int D>
 cudaError_t launch_d(const AttnArgs& a, cudaStream_t s) {
-  const bool rope = a.rope_cos != nullptr;
-  if (two_tiles(a)) return rope ? launch_tc<BITS, D, 2, true>(a, s) : launch_tc<BITS, D, 2, false>(a, s);
-  return rope ? launch_tc<BITS, D, 1, true>(a, s) : launch_tc<BITS, D, 1, false>(a, s);
+  if (has_rope(a)) {
+    if constexpr (D == 64) {
+      if (a.kv_split) return launch_tc<BITS, D, 1, true>(a, s);
+    }
+    return cudaErrorInvalidConfiguration;
+  }
+  return two_tiles(a) ? launch_tc<BITS, D, 2, false>(a, s) : launch_tc<BITS, D, 1, false>(a, s);
 }
 
 template <int BITS>
@@ -344,14 +346,14 @@ cudaError_t launch_bits(const AttnArgs& a, cudaStream_t s) {
 // per-tile chain softmax -> P V -> Q K^T is the bottleneck (no RoPE, and the
 // split-KV form with one query tile per CTA) the single-CTA kernel is faster:
 // the pair's cross-CTA signals lengthen that chain.
-bool use_pair_kernel(const AttnArgs& a) { return a.rope_cos != nullptr && !a.kv_split; }
+bool use_pair_kernel(const AttnArgs& a) { return has_rope(a) && !a.kv_split; }
 
 // Split-KV form: enough CTAs for about two waves over 148 SMs (one CTA per
 // SM), each range at least four KV tiles long when the cache allows, and no
 // empty range; then, up to twice that many ranges, the count that fills the
 // last wave best.
 int split_kv_splits(const AttnArgs& a) {
-  const int nkv = tile_tokens(a.bits);
+  const int nkv = kv_tile_tokens(a.bits);
   const int ntiles = (a.t_att + nkv - 1) / nkv;
   const int64_t base = int64_t((a.lq + BM - 1) / BM) * a.heads * a.batch;  // single-CTA kernel
   int64_t want = (2 * 148 + base - 1) / base;

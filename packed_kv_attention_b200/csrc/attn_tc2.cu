@@ -84,6 +84,7 @@ struct Cfg2 {
   static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
   static_assert(NKV % 16 == 0 && NKV <= 128 && HALF <= 64, "tile shape");
   static_assert(HALF % GT == 0 && NW % 2 == 0, "each CTA's K half is whole groups of whole words");
+  static_assert(GT == dequant_group_tokens(BITS), "rotary table rows assume the host's group size");
 };
 
 constexpr int kRelayWarp = 18;
@@ -155,6 +156,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   if constexpr (ROPE)
     rope_key_bound_partial<BITS, D, kThreads2>(a.k_meta + (int64_t(b) * a.heads + h) * a.n_blocks_total * D,
                                                a.n_cached_blocks, bars);
+  // rotary mode 2: the CTA's table of the 3D schedule, after the barrier
+  // region (both CTAs of the pair cover the same tiles)
+  float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
+  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * C::NKV) / a.rope_frame : 0;
+  if constexpr (ROPE)
+    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kThreads2);
   // query tiles -> K-major swizzled smem (rows past lq are zero).  The CH
   // chunks of a row are consecutive lanes of one warp in one pass, so with
   // fp16 operands they agree on the row's exponent by shuffles.
@@ -311,6 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     // (row dv of the V tile = channel rank D/2 + dv, groups from partv)
     const int dt = tid - kDequantWarp0 * 32;
     const int dk = dt % D, partk = dt / D;
+    const RopeTable rtab = rope_table_of(a, rope_tab, dk, rope_f0);  // rotary mode 2 (keys only)
     const int dv = dt % C::DH, partv = dt / C::DH;
     const int64_t bh = int64_t(b) * a.heads + h;
     const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + dk;
@@ -411,22 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               x[jt] = v;
             }
           }
-          if (ROPE && tensor == 0) {
-            // pre-RoPE key mode: rotate pair (2i, 2i+1) of every token after
-            // dequantization; the partner channel lives in the neighbour lane
-#pragma unroll
-            for (int jt = 0; jt < C::GT; ++jt) {
-              const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
-              const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
-              const int t = tg + jt;
-              float c = 1.0f, s = 0.0f;
-              if (t < t_att) {
-                c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
-                s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
-              }
-              x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
-            }
-          }
+          if (ROPE && tensor == 0) rope_rotate<C::GT, D>(a, rtab, x, tg, d);
 #pragma unroll
           for (int c = 0; c < C::GC; ++c) {
             uint32_t pk[4];
@@ -647,11 +640,13 @@ template <int BITS, int D, int NQ, bool ROPE>
 cudaError_t launch_tc2(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg2<BITS, D, NQ>;
   auto kern = attn_tc2_kernel<BITS, D, NQ, ROPE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+  const uint32_t smem = C::SMEM + (ROPE ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
+  if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int pairs = (a.lq + 2 * NQ * BM - 1) / (2 * NQ * BM) * (a.kv_split ? a.n_splits : 1);
   dim3 grid(unsigned(2 * pairs), a.heads, a.batch);
-  kern<<<grid, kThreads2, C::SMEM, stream>>>(a);
+  kern<<<grid, kThreads2, smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || !a.kv_split) return e;
   return launch_attention_combine(a, stream);
@@ -666,7 +661,7 @@ bool pair_two_tiles(const AttnArgs& a) {
 
 template <int BITS, int D>
 cudaError_t launch_d2(const AttnArgs& a, cudaStream_t s) {
-  const bool rope = a.rope_cos != nullptr;
+  const bool rope = has_rope(a);
   if (pair_two_tiles(a)) return rope ? launch_tc2<BITS, D, 2, true>(a, s) : launch_tc2<BITS, D, 2, false>(a, s);
   return rope ? launch_tc2<BITS, D, 1, true>(a, s) : launch_tc2<BITS, D, 1, false>(a, s);
 }

@@ -17,6 +17,7 @@ constexpr int kMmaWarp = 17;
 constexpr int BM = 128;
 constexpr float kRescaleThreshold = 16.0f;  // log2 units
 constexpr uint32_t kSmemUsable = 227 * 1024 - 1024;  // minus 1 KB to align the base to 1024
+constexpr uint32_t kSmemMaxDynamic = 227 * 1024;      // dynamic shared memory of one CTA
 constexpr uint32_t kBarBytes = 2048;
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
@@ -383,6 +384,155 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
 }
 
 
+
+// ------------------------------------------------------------------ 3D RoPE
+// Rotary mode 2: token t lies in frame f = t / frame, at row (t % frame) /
+// gw and column t % gw; key pair i belongs to the frame axis (i < P0), the
+// row axis (i < P0 + P1) or the column axis, as pair j of that axis's n, and
+// turns by pos * base^(-j / n) radians (project page, "The block axis", Eq. 3:
+// RoPE rotates each (2i, 2i+1) key pair; the 3D frame/row/column schedule of
+// the video models).  Each CTA tabulates cos and sin of every angle its
+// tokens use, computed in double precision and rounded to fp32 as a host
+// table would be.  Layout: per pair, its axis's positions in a row of
+// rope_len[axis] float2 entries -- frames f0, f0 + 1, ..., rows 0, 1, ...
+// (entry r holds row r mod rows), columns 0, 1, ... (entry c holds c mod gw),
+// each running on past the CTA's last frame, the last row and the last column
+// as far as one dequant group of GT tokens reaches -- so that a group reads
+// entries col + j (columns) and pos, pos + 1, ... (rows, frames) without a
+// wrap test.
+
+__device__ __forceinline__ int div_magic_dev(int t, uint32_t m, int s) {
+  return int((uint64_t(uint32_t(t)) * m) >> s);
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// Fill the table (all threads of the CTA; a __syncthreads must follow).
+__device__ __forceinline__ void rope_table_build(const AttnArgs& a, float2* tab, int f0, int nthreads) {
+  const int p0 = a.rope_pairs[0], p1 = a.rope_pairs[1], p2 = a.rope_pairs[2];
+  const int l0 = a.rope_len[0], l1 = a.rope_len[1], l2 = a.rope_len[2];
+  const int n0 = p0 * l0, n1 = p1 * l1, n2 = p2 * l2;
+  const double lb = log2(double(a.rope_base));
+  for (int e = threadIdx.x; e < n0 + n1 + n2; e += nthreads) {
+    int pos, j, n;
+    if (e < n0) {
+      j = e / l0, pos = f0 + e % l0, n = p0;
+    } else if (e < n0 + n1) {
+      j = (e - n0) / l1, pos = (e - n0) % l1 % a.rope_rows, n = p1;
+    } else {
+      j = (e - n0 - n1) / l2, pos = (e - n0 - n1) % l2 % a.rope_gw, n = p2;
+    }
+    const double ang = double(pos) * exp2(-double(j) / double(n) * lb);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    tab[e] = make_float2(float(cs), float(sn));
+  }
+}
+
+// This thread's row of the table for key channel d (pair d / 2).
+struct RopeTable {
+  uint32_t row;  // shared address of the pair's first entry
+  int axis;      // 0 frame, 1 row, 2 column
+  int f0;        // first frame of the table
+};
+
+__device__ __forceinline__ RopeTable rope_table_of(const AttnArgs& a, const float2* tab, int d, int f0) {
+  const int i = d >> 1, p0 = a.rope_pairs[0], p1 = a.rope_pairs[1];
+  const int l0 = a.rope_len[0], l1 = a.rope_len[1], l2 = a.rope_len[2];
+  RopeTable r;
+  r.f0 = f0;
+  int e;
+  if (i < p0) {
+    r.axis = 0, e = i * l0;
+  } else if (i < p0 + p1) {
+    r.axis = 1, e = p0 * l0 + (i - p0) * l1;
+  } else {
+    r.axis = 2, e = p0 * l0 + p1 * l1 + (i - p0 - p1) * l2;
+  }
+  r.row = smem_u32(tab) + uint32_t(e) * 8u;
+  return r;
+}
+
+// Pre-RoPE key mode: rotate pair (2i, 2i+1) of the GT dequantized values of
+// channel d, tokens tg .. tg + GT - 1, after rounding them to bf16 (the value
+// the cache would hold); the partner channel lives in the neighbour lane.
+// Rotation angles come from the caller's [T][D/2] tables (mode 1) or from the
+// CTA's table of the 3D schedule (mode 2).  Values past the attended tokens
+// are zero and stay zero.  tg is the same in every lane of the warp.
+template <int GT, int D>
+__device__ __forceinline__ void rope_rotate(const AttnArgs& a, const RopeTable& r, float (&x)[GT], int tg, int d) {
+  const int t_att = a.t_att;
+  if (a.rope_mode != 2) {
+#pragma unroll
+    for (int jt = 0; jt < GT; ++jt) {
+      const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
+      const int t = tg + jt;
+      float c = 1.0f, s = 0.0f;
+      if (t < t_att) {
+        c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
+        s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
+      }
+      x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
+    }
+    return;
+  }
+  if (tg >= t_att) return;
+  const int f = div_magic_dev(tg, a.rope_frame_mul, a.rope_frame_shift);
+  const int p = tg - f * a.rope_frame;
+  const int row = div_magic_dev(p, a.rope_gw_mul, a.rope_gw_shift);
+  const int col = p - row * a.rope_gw;
+  if (a.rope_gw >= GT) {
+    // the group crosses at most one row (and frame) boundary: columns read
+    // entries col + jt, rows and frames entry pos up to token jb, pos + 1 on
+    uint32_t addr;
+    int inc, jb;
+    if (r.axis == 2) {
+      addr = r.row + uint32_t(col) * 8u, inc = 8, jb = GT;
+    } else if (r.axis == 1) {
+      addr = r.row + uint32_t(row) * 8u, inc = 0, jb = a.rope_gw - col;
+    } else {
+      addr = r.row + uint32_t(f - r.f0) * 8u, inc = 0, jb = a.rope_frame - p;
+    }
+#pragma unroll
+    for (int jt = 0; jt < GT; ++jt) {
+      const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
+      const float2 cs = lds_f2(addr + uint32_t(jt * inc) + (jt >= jb ? 8u : 0u));
+      x[jt] = (d & 1) ? __fmaf_rn(other, cs.y, xr * cs.x) : __fmaf_rn(-other, cs.y, xr * cs.x);
+    }
+  } else {
+    // rows narrower than a group: count down to each row (frame) boundary;
+    // the row and frame entries run on past the last row / frame as far as
+    // one group reaches, so positions never wrap
+    int idx, inc, cnt, period;
+    if (r.axis == 2) {
+      idx = col, inc = 1, cnt = GT + 1, period = 0;
+    } else if (r.axis == 1) {
+      idx = row, inc = 0, cnt = a.rope_gw - col, period = a.rope_gw;
+    } else {
+      idx = f - r.f0, inc = 0, cnt = a.rope_frame - p, period = a.rope_frame;
+    }
+#pragma unroll
+    for (int jt = 0; jt < GT; ++jt) {
+      const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
+      if (cnt == 0) {
+        ++idx;
+        cnt = period;
+      }
+      const float2 cs = lds_f2(r.row + uint32_t(idx) * 8u);
+      x[jt] = (d & 1) ? __fmaf_rn(other, cs.y, xr * cs.x) : __fmaf_rn(-other, cs.y, xr * cs.x);
+      idx += inc;
+      --cnt;
+    }
+  }
+}
+
 // The dequant warps of the single-CTA tensor-core kernels.  Thread dt owns
 // channel d = dt % D and the dequant groups part, part + TPC, ... of every KV
 // tile (a group = GT tokens = whole packed words and whole 16-byte chunks).
@@ -403,10 +553,12 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
 // dequant threads, the arrival count of kready/vready/empty).
 template <class C, int BITS, int D, bool ROPE>
 __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, uint8_t* smem, const int* sm_bs, int dt,
-                                             int b, int h, int tile0, int ntiles, int kexp) {
+                                             int b, int h, int tile0, int ntiles, int kexp, const float2* rope_tab,
+                                             int rope_f0) {
   constexpr int CPW = C::CPW;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   constexpr bool QK_F16 = ROPE;
+  static_assert(C::GT == dequant_group_tokens(BITS), "rotary table rows assume the host's group size");
   volatile int* abort_flag = &bars->abort_flag;
   const int t_att = a.t_att;
   const int d = dt % D;
@@ -415,6 +567,7 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
   const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + d;
   const uint32_t* mgv = a.v_meta + bh * a.n_blocks_total * D + d;
   const int nblk = a.n_cached_blocks;
+  const RopeTable rtab = rope_table_of(a, rope_tab, d, rope_f0);  // rotary mode 2
   // (scale, min) words of this thread's channel for block blk and blk + 1,
   // K and V, loaded one block ahead so a tile never waits on them
   uint32_t mk_cur = __ldg(mgk), mv_cur = __ldg(mgv);
@@ -511,22 +664,7 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
             x[jt] = v;
           }
         }
-        if (ROPE && tensor == 0) {
-          // pre-RoPE key mode: rotate pair (2i, 2i+1) of every token after
-          // dequantization; the partner channel lives in the neighbour lane
-#pragma unroll
-          for (int jt = 0; jt < C::GT; ++jt) {
-            const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
-            const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
-            const int t = tg + jt;
-            float c = 1.0f, s = 0.0f;
-            if (t < t_att) {
-              c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
-              s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
-            }
-            x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
-          }
-        }
+        if (ROPE && tensor == 0) rope_rotate<C::GT, D>(a, rtab, x, tg, d);
 #pragma unroll
         for (int c = 0; c < C::GC; ++c) {
           uint32_t pk[4];

@@ -99,6 +99,18 @@ struct AttnArgs {
   int32_t kv_split;        // 1: each CTA attends to one of n_splits ranges of KV tiles and writes an
                            // unnormalised partial (O, m, l) to the workspace; a combine kernel merges them
   int32_t n_splits;
+  // pre-RoPE key mode: 0 none, 1 caller tables (rope_cos, rope_sin), 2 a 3D
+  // rotary schedule whose angles each CTA computes (frame, row, column axes)
+  int32_t rope_mode;
+  int32_t rope_frame;      // tokens per frame (rope_rows * rope_gw)
+  int32_t rope_gw;         // tokens per row
+  int32_t rope_rows;       // rows per frame
+  int32_t rope_pairs[3];   // rotary pairs of the frame, row and column axes (sum D/2)
+  float rope_base;
+  int32_t rope_frames;     // frames a CTA's tokens can span (the most any CTA's KV range does)
+  int32_t rope_len[3];     // table entries per pair along the frame, row and column axes (odd)
+  uint32_t rope_frame_mul, rope_gw_mul;  // t / rope_frame == (t * mul) >> shift for 0 <= t < 2^30
+  int32_t rope_frame_shift, rope_gw_shift;
   int32_t block_start[VARQ_MAX_BLOCKS + 1];
 };
 
@@ -108,6 +120,64 @@ struct DenseTensor {
   const void* ptr;
   int64_t sb, sh, st;
 };
+
+inline bool has_rope(const AttnArgs& a) { return a.rope_mode != 0; }
+// Tokens per KV tile of the packed-cache attention kernels for a bit width:
+// whole words of whole 16-token MMA slices, at most 128 (128, 96 for 5-bit, 80
+// for 3- and 6-bit).
+inline int kv_tile_tokens(int bits) {
+  const int cpw = 32 / bits;
+  int g = cpw, h = 16;
+  while (h != 0) {
+    const int t = g % h;
+    g = h;
+    h = t;
+  }
+  const int unit = cpw / g * 16;
+  return (128 / unit) * unit;
+}
+// Tokens per dequant group of those kernels: whole packed words and whole
+// 8-token (16-byte) chunks, lcm(32 / bits, 8).
+constexpr int dequant_group_tokens(int bits) {
+  const int cpw = 32 / bits;
+  int g = cpw, h = 8;
+  while (h != 0) {
+    const int t = g % h;
+    g = h;
+    h = t;
+  }
+  return cpw / g * 8;
+}
+// Division by a positive divisor d as a multiply and a shift, exact for
+// 0 <= t < 2^30: s = 30 + ceil(log2 d), m = ceil(2^s / d) <= 2^31 (the
+// round-up method of Granlund and Montgomery, "Division by invariant integers
+// using multiplication", 1994: m d - 2^s < d bounds the error below 1/d).
+inline void div_magic(int d, uint32_t& m, int32_t& s) {
+  int l = 0;
+  while ((int64_t(1) << l) < d) ++l;
+  s = 30 + l;
+  m = static_cast<uint32_t>(((uint64_t(1) << s) + uint64_t(d) - 1) / uint64_t(d));
+}
+// Per-pair row lengths of the rotary table of rope_mode 2 (rope_frames,
+// rope_rows and rope_gw set): a group of GT tokens that starts in the last
+// frame, row or column reaches (frame - 1 + GT - 1) / frame frames,
+// (gw - 1 + GT - 1) / gw rows and GT - 1 columns further, so each axis runs
+// on that far; each length is rounded up to odd so that the 16 pairs one warp
+// reads fall in distinct shared-memory banks.
+inline void set_rope_lens(AttnArgs& a) {
+  const int gt = dequant_group_tokens(a.bits);
+  a.rope_len[0] = (a.rope_frames + (a.rope_frame + gt - 2) / a.rope_frame) | 1;
+  a.rope_len[1] = (a.rope_rows + (a.rope_gw + gt - 2) / a.rope_gw) | 1;
+  a.rope_len[2] = (a.rope_gw + gt - 1) | 1;
+}
+// Bytes of the per-CTA rotary table of rope_mode 2 (0 otherwise): float2
+// (cos, sin) entries, per pair, along its axis.
+inline uint32_t rope_table_bytes(const AttnArgs& a) {
+  if (a.rope_mode != 2) return 0;
+  const int64_t n = int64_t(a.rope_len[0]) * a.rope_pairs[0] + int64_t(a.rope_len[1]) * a.rope_pairs[1] +
+                    int64_t(a.rope_len[2]) * a.rope_pairs[2];
+  return uint32_t(((n * 8) + 127) / 128 * 128);
+}
 
 // Tensor-core attention; with kv_split, the split-KV form plus its combine.
 // Pre-RoPE keys on the tensor path go to the paired-CTA kernel

@@ -167,18 +167,61 @@ size_t varq_packed_attention_workspace(const varq_cache_layout* L, int lq, int n
   return varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, n);
 }
 
-int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st,
-                          int lq, const uint32_t* k_packed, const uint32_t* k_meta, const uint32_t* v_packed,
-                          const uint32_t* v_meta, int n_cached_blocks, float softmax_scale, const float* rope_cos,
-                          const float* rope_sin, void* out, int64_t o_sb, int64_t o_sh, int64_t o_st, float* lse,
-                          void* workspace, size_t workspace_bytes, int path, uint32_t* dev_status, void* stream) {
+// Path choice, split-KV workspace check and launch of a filled argument block
+// (shared by the table and the 3D-schedule rotary entry points).
+static int run_attention(const varq_cache_layout* L, AttnArgs& a, void* workspace, size_t workspace_bytes, int path,
+                         cudaStream_t s) {
+  const int p = choose_path(a.lq, path);
+  if (p == VARQ_PATH_SPLIT && a.lq > VARQ_SPLIT_MAX_LQ) return VARQ_ERR_UNSUPPORTED;
+  if (p == VARQ_PATH_SPLIT) a.kv_split = 1;
+  const bool dec = p == VARQ_PATH_SPLIT && varq::use_decode_kernel(a);
+  if (p == VARQ_PATH_SPLIT) {
+    // ranges of the cache over CTAs (the CUDA-core kernel on the packed codes,
+    // or a tensor-core kernel with pre-RoPE keys), then the merge
+    a.n_splits = dec ? varq::split_kv_decode_splits(a) : varq::split_kv_splits(a);
+    const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, a.lq, L->head_dim, a.n_splits);
+    if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
+    a.workspace = static_cast<float*>(workspace);
+  }
+  if (a.rope_mode == 2) {
+    // frames of the schedule a CTA's tokens can span: all of them, or those of
+    // one split range
+    const int64_t frames_all = (int64_t(a.t_att) + a.rope_frame - 1) / a.rope_frame;
+    int64_t frames = frames_all;
+    if (a.kv_split) {
+      const int nkv = varq::kv_tile_tokens(a.bits);
+      const int64_t per = (int64_t(a.t_att) + nkv - 1) / nkv;
+      const int64_t span = (per + a.n_splits - 1) / a.n_splits * nkv;
+      frames = std::min<int64_t>(frames_all, (span + a.rope_frame - 1) / a.rope_frame + 1);
+    }
+    a.rope_frames = static_cast<int32_t>(frames);
+    varq::set_rope_lens(a);
+  }
+  cudaError_t e;
+  if (p == VARQ_PATH_TENSOR)
+    e = varq::launch_attention_tc(a, s);
+  else if (dec)
+    e = varq::launch_attention_decode(a, s);
+  else
+    e = varq::use_swap_ab_kernel(a) ? varq::launch_attention_swap_ab(a, s) : varq::launch_attention_tc(a, s);
+  // a rotary table that does not fit in shared memory next to the kernel's buffers
+  if (e == cudaErrorInvalidConfiguration) return VARQ_ERR_UNSUPPORTED;
+  return launch_status(e);
+}
+
+// Checks and argument block common to both attention entry points.
+static int prepare_attention(AttnArgs& a, const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh,
+                             int64_t q_st, int lq, const uint32_t* k_packed, const uint32_t* k_meta,
+                             const uint32_t* v_packed, const uint32_t* v_meta, int n_cached_blocks, float softmax_scale,
+                             void* out, int64_t o_sb, int64_t o_sh, int64_t o_st, float* lse, int path,
+                             uint32_t* dev_status) {
   int rc = check_layout(L);
   if (rc != VARQ_OK) return rc;
   if (q == nullptr || out == nullptr || k_packed == nullptr || k_meta == nullptr || v_packed == nullptr ||
       v_meta == nullptr)
     return VARQ_ERR_INVALID_ARG;
   if (lq < 1 || n_cached_blocks < 1 || n_cached_blocks > L->n_blocks) return VARQ_ERR_INVALID_ARG;
-  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return VARQ_ERR_INVALID_ARG;
   if (path != VARQ_PATH_AUTO && path != VARQ_PATH_TENSOR && path != VARQ_PATH_SPLIT) return VARQ_ERR_INVALID_ARG;
   if (!(std::isfinite(softmax_scale))) return VARQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(k_meta) || !aligned16(v_packed) ||
@@ -188,10 +231,6 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
       !stride_ok(o_st))
     return VARQ_ERR_ALIGNMENT;
   if (L->heads > 65535 || L->batch > 65535) return VARQ_ERR_UNSUPPORTED;
-  const int p = choose_path(lq, path);
-  if (p == VARQ_PATH_SPLIT && lq > VARQ_SPLIT_MAX_LQ) return VARQ_ERR_UNSUPPORTED;
-
-  AttnArgs a;
   fill_attn(a, L, lq, n_cached_blocks);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.q_sb = q_sb;
@@ -201,8 +240,6 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   a.k_meta = k_meta;
   a.v_packed = v_packed;
   a.v_meta = v_meta;
-  a.rope_cos = rope_cos;
-  a.rope_sin = rope_sin;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.o_sb = o_sb;
   a.o_sh = o_sh;
@@ -212,21 +249,51 @@ int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_s
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(float(L->head_dim));
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p == VARQ_PATH_TENSOR) return launch_status(varq::launch_attention_tc(a, s));
+  return VARQ_OK;
+}
 
-  // split-KV form: ranges of the cache over CTAs (the CUDA-core kernel on the
-  // packed codes, or the tensor-core kernel with pre-RoPE keys), then the merge
-  a.kv_split = 1;
-  const bool dec = varq::use_decode_kernel(a);
-  a.n_splits = dec ? varq::split_kv_decode_splits(a) : varq::split_kv_splits(a);
-  const size_t need = varq::split_kv_workspace_bytes(L->batch, L->heads, lq, L->head_dim, a.n_splits);
-  if (workspace == nullptr || workspace_bytes < need) return VARQ_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return VARQ_ERR_ALIGNMENT;
-  a.workspace = static_cast<float*>(workspace);
-  if (dec) return launch_status(varq::launch_attention_decode(a, s));
-  return launch_status(varq::use_swap_ab_kernel(a) ? varq::launch_attention_swap_ab(a, s)
-                                                   : varq::launch_attention_tc(a, s));
+int varq_packed_attention(const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st,
+                          int lq, const uint32_t* k_packed, const uint32_t* k_meta, const uint32_t* v_packed,
+                          const uint32_t* v_meta, int n_cached_blocks, float softmax_scale, const float* rope_cos,
+                          const float* rope_sin, void* out, int64_t o_sb, int64_t o_sh, int64_t o_st, float* lse,
+                          void* workspace, size_t workspace_bytes, int path, uint32_t* dev_status, void* stream) {
+  AttnArgs a;
+  int rc = prepare_attention(a, L, q, q_sb, q_sh, q_st, lq, k_packed, k_meta, v_packed, v_meta, n_cached_blocks,
+                             softmax_scale, out, o_sb, o_sh, o_st, lse, path, dev_status);
+  if (rc != VARQ_OK) return rc;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return VARQ_ERR_INVALID_ARG;
+  a.rope_cos = rope_cos;
+  a.rope_sin = rope_sin;
+  a.rope_mode = rope_cos != nullptr ? 1 : 0;
+  return run_attention(L, a, workspace, workspace_bytes, path, static_cast<cudaStream_t>(stream));
+}
+
+int varq_packed_attention_rope3d(const varq_cache_layout* L, const void* q, int64_t q_sb, int64_t q_sh, int64_t q_st,
+                                 int lq, const uint32_t* k_packed, const uint32_t* k_meta, const uint32_t* v_packed,
+                                 const uint32_t* v_meta, int n_cached_blocks, float softmax_scale,
+                                 const varq_rope3d* rope, void* out, int64_t o_sb, int64_t o_sh, int64_t o_st,
+                                 float* lse, void* workspace, size_t workspace_bytes, int path, uint32_t* dev_status,
+                                 void* stream) {
+  AttnArgs a;
+  int rc = prepare_attention(a, L, q, q_sb, q_sh, q_st, lq, k_packed, k_meta, v_packed, v_meta, n_cached_blocks,
+                             softmax_scale, out, o_sb, o_sh, o_st, lse, path, dev_status);
+  if (rc != VARQ_OK) return rc;
+  if (rope == nullptr) return VARQ_ERR_INVALID_ARG;
+  if (rope->grid_w < 1 || rope->frame_tokens < rope->grid_w || rope->frame_tokens % rope->grid_w != 0)
+    return VARQ_ERR_INVALID_ARG;
+  if (rope->pairs[0] < 0 || rope->pairs[1] < 0 || rope->pairs[2] < 0 ||
+      rope->pairs[0] + rope->pairs[1] + rope->pairs[2] != L->head_dim / 2)
+    return VARQ_ERR_INVALID_ARG;
+  if (!(rope->base > 0.0f) || !std::isfinite(rope->base)) return VARQ_ERR_INVALID_ARG;
+  a.rope_mode = 2;
+  a.rope_frame = rope->frame_tokens;
+  a.rope_gw = rope->grid_w;
+  a.rope_rows = rope->frame_tokens / rope->grid_w;
+  varq::div_magic(a.rope_frame, a.rope_frame_mul, a.rope_frame_shift);
+  varq::div_magic(a.rope_gw, a.rope_gw_mul, a.rope_gw_shift);
+  for (int i = 0; i < 3; ++i) a.rope_pairs[i] = rope->pairs[i];
+  a.rope_base = rope->base;
+  return run_attention(L, a, workspace, workspace_bytes, path, static_cast<cudaStream_t>(stream));
 }
 
 static int check_dense(int batch, int heads, int head_dim, int64_t n_tokens, int lq, int path) {

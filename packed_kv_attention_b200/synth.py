@@ -33,7 +33,7 @@ import torch
 
 __all__ = [
     "Workload", "WORKLOADS", "block_starts", "kv_cache", "queries",
-    "rope_tables_3d", "make_inputs",
+    "rope_tables_3d", "rope_axis_pairs", "make_inputs",
 ]
 
 
@@ -127,6 +127,12 @@ def queries(gen: torch.Generator, batch: int, heads: int, lq: int, head_dim: int
                        dtype=torch.float32).to(torch.bfloat16)
 
 
+def rope_axis_pairs(head_dim: int) -> Tuple[int, int, int]:
+    """Rotary pairs of the (frame, row, column) axes: 64 pairs -> 22:21:21."""
+    pairs = head_dim // 2
+    return (pairs - 2 * (pairs // 3), pairs // 3, pairs // 3)
+
+
 def rope_tables_3d(n_tokens: int, head_dim: int, chunk: int = 4680, frame: int = 1560,
                    grid_w: int = 52, split: Optional[Tuple[int, int, int]] = None,
                    base: float = 10000.0, device="cpu") -> Tuple[torch.Tensor, torch.Tensor]:
@@ -140,8 +146,7 @@ def rope_tables_3d(n_tokens: int, head_dim: int, chunk: int = 4680, frame: int =
     """
     pairs = head_dim // 2
     if split is None:
-        a = pairs - 2 * (pairs // 3)
-        split = (a, pairs // 3, pairs // 3)   # 64 pairs -> 22:21:21
+        split = rope_axis_pairs(head_dim)     # 64 pairs -> 22:21:21
     assert sum(split) == pairs
     t = torch.arange(n_tokens, dtype=torch.float64, device=device)
     ci = torch.div(t, chunk, rounding_mode="floor")

@@ -20,7 +20,7 @@ __all__ = [
     "PATH_AUTO", "PATH_TENSOR", "PATH_SPLIT", "SPLIT_MAX_LQ",
     "DEV_NONFINITE", "DEV_META_OVERFLOW", "DEV_TIMEOUT",
     "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "varq_quantize_pack_launches",
-    "varq_dense_attention", "varq_dense_attention_workspace",
+    "varq_dense_attention", "varq_dense_attention_workspace", "Rope3d", "varq_packed_attention_rope3d",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvarq.so")
@@ -55,6 +55,20 @@ class CacheLayout(ctypes.Structure):
     def __repr__(self):
         return (f"CacheLayout(B={self.batch}, H={self.heads}, D={self.head_dim}, bits={self.bits}, "
                 f"NB={self.n_blocks}, T={self.n_tokens}, W={self.words_per_row})")
+
+
+class Rope3d(ctypes.Structure):
+    """Mirror of ``varq_rope3d``: the 3D (frame, row, column) rotary schedule."""
+    _fields_ = [("frame_tokens", ctypes.c_int32), ("grid_w", ctypes.c_int32), ("pairs", ctypes.c_int32 * 3),
+                ("base", ctypes.c_float)]
+
+    @classmethod
+    def make(cls, frame_tokens: int, grid_w: int, pairs: Sequence[int], base: float = 10000.0) -> "Rope3d":
+        r = cls()
+        r.frame_tokens, r.grid_w, r.base = int(frame_tokens), int(grid_w), float(base)
+        for i in range(3):
+            r.pairs[i] = int(pairs[i])
+        return r
 
 
 _LIB = None
@@ -93,6 +107,11 @@ def lib() -> ctypes.CDLL:
             _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_f,
             _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_int, _c_p, _c_p]
         L.varq_dense_attention.restype = _c_int
+        L.varq_packed_attention_rope3d.argtypes = [
+            ctypes.POINTER(CacheLayout), _c_p, _c_i64, _c_i64, _c_i64, _c_int,
+            _c_p, _c_p, _c_p, _c_p, _c_int, _c_f, ctypes.POINTER(Rope3d),
+            _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_int, _c_p, _c_p]
+        L.varq_packed_attention_rope3d.restype = _c_int
         L.varq_status_string.argtypes = [_c_int]
         L.varq_status_string.restype = ctypes.c_char_p
         L.varq_abi_version.argtypes = []
@@ -292,3 +311,30 @@ def varq_dense_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out:
         float(softmax_scale), _ptr(out), out.stride(0), out.stride(1), out.stride(2), _ptr(lse), _ptr(workspace),
         ws_bytes, path, _ptr(dev_status), _stream(stream))
     _check(rc, "varq_dense_attention")
+
+
+def varq_packed_attention_rope3d(layout: CacheLayout, q: torch.Tensor, k_packed: torch.Tensor, k_meta: torch.Tensor,
+                                 v_packed: torch.Tensor, v_meta: torch.Tensor, out: torch.Tensor, rope: Rope3d,
+                                 n_cached_blocks: Optional[int] = None, softmax_scale: float = 0.0,
+                                 lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                                 path: int = PATH_AUTO, dev_status: Optional[torch.Tensor] = None,
+                                 stream=None) -> None:
+    """Pre-RoPE key attention with the rotation angles computed in the kernel
+    from the 3D schedule ``rope`` (a ``Rope3d``) instead of tables."""
+    if n_cached_blocks is None:
+        n_cached_blocks = layout.n_blocks
+    _need(q, "q", torch.bfloat16)
+    _need(out, "out", torch.bfloat16)
+    for t, n in ((k_packed, "k_packed"), (k_meta, "k_meta"), (v_packed, "v_packed"), (v_meta, "v_meta")):
+        _need(t, n)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    if q.dim() != 4 or q.stride(3) != 1 or out.dim() != 4 or out.stride(3) != 1:
+        raise ValueError("q and out must be [B, H, lq, D] with contiguous channels")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().varq_packed_attention_rope3d(
+        ctypes.byref(layout), _ptr(q), q.stride(0), q.stride(1), q.stride(2), q.shape[2],
+        _ptr(k_packed), _ptr(k_meta), _ptr(v_packed), _ptr(v_meta), n_cached_blocks, float(softmax_scale),
+        ctypes.byref(rope), _ptr(out), out.stride(0), out.stride(1), out.stride(2),
+        _ptr(lse), _ptr(workspace), ws_bytes, path, _ptr(dev_status), _stream(stream))
+    _check(rc, "varq_packed_attention_rope3d")

@@ -157,6 +157,35 @@ def test_attention_errors():
     assert V.varq_packed_attention_workspace(L, 4, 3, V.PATH_TENSOR) == 0
 
 
+def test_rope3d_attention_errors():
+    lib = V.lib()
+    L = _layout()
+    P = ctypes.c_void_p
+
+    def call(frame=40, gw=8, pairs=(22, 21, 21), base=10000.0, lq=64, nc=3, rope=True, q=FAKE, path=0, lay=L):
+        r = V.Rope3d.make(frame, gw, pairs, base)
+        return lib.varq_packed_attention_rope3d(ctypes.byref(lay), P(q), 8, 8, 128, lq, P(FAKE), P(FAKE), P(FAKE),
+                                                P(FAKE), nc, 0.0, ctypes.byref(r) if rope else None, P(FAKE), 8, 8,
+                                                128, None, None, 0, path, None, None)
+
+    assert call(rope=False) == INVALID
+    assert call(gw=0) == INVALID
+    assert call(frame=4, gw=8) == INVALID        # frame shorter than one grid row
+    assert call(frame=42, gw=8) == INVALID       # frame not a whole number of rows
+    assert call(pairs=(22, 21, 20)) == INVALID   # pairs must cover D/2 = 64
+    assert call(pairs=(-1, 33, 32)) == INVALID
+    assert call(base=0.0) == INVALID
+    assert call(base=float("inf")) == INVALID
+    assert call(base=float("nan")) == INVALID
+    assert call(lq=0) == INVALID                 # the common checks still apply
+    assert call(q=FAKE + 2) == ALIGN
+    assert call(lq=4) == WORKSPACE
+    # a schedule of one-token frames has more frame angles than shared memory
+    # holds next to the kernel's buffers: refused before any launch
+    long_cache = V.varq_cache_alloc(1, 1, 128, 4, [0, 50000, 100000])
+    assert call(frame=1, gw=1, path=1, nc=2, lay=long_cache) == UNSUPPORTED
+
+
 def test_dense_attention_errors():
     lib = V.lib()
     P = ctypes.c_void_p
