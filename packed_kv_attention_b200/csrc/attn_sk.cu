@@ -117,7 +117,7 @@ __device__ __forceinline__ float ord2f(uint32_t u) {
 
 }  // namespace
 
-template <int BITS, bool ROPE>
+template <int BITS, bool ROPE, bool SCHED>
 __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_constant__ AttnArgs a) {
   constexpr int D = 128;
   using C = SkCfg<BITS, D>;
@@ -176,9 +176,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
                                                 a.n_cached_blocks, bars);
   // rotary mode 2: the CTA's table of the 3D schedule, after the barrier region
   float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
-  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * NKV) / a.rope_frame : 0;
-  if constexpr (ROPE)
-    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kSkThreads);
+  const int rope_f0 = SCHED ? (tile0 * NKV) / a.rope_frame : 0;
+  if constexpr (SCHED) rope_table_build(a, rope_tab, rope_f0, kSkThreads);
   // the 16-row query tile -> K-major swizzled smem (rows past lq are zero);
   // a row's 16 chunks are lanes 0-15 or 16-31 of one warp
   {
@@ -261,7 +260,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     }
   } else if (warp >= kSkDeqWarp0) {
     // ------------------------------------------------------------- dequant
-    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, tid - kSkDeqWarp0 * 32, b, h, tile0, ntiles, kexp, rope_tab,
+    dequant_loop<C, BITS, D, ROPE, SCHED>(a, bars, smem, sm_bs, tid - kSkDeqWarp0 * 32, b, h, tile0, ntiles, kexp, rope_tab,
                                    rope_f0);
   } else {
     // ------------------------------------------------------------- softmax
@@ -425,11 +424,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
 
 namespace {
 
-template <int BITS, bool ROPE>
+template <int BITS, bool ROPE, bool SCHED = false>
 cudaError_t launch_sk(const AttnArgs& a, cudaStream_t stream) {
   using C = SkCfg<BITS, 128>;
-  auto kern = attn_sk_kernel<BITS, ROPE>;
-  const uint32_t smem = C::SMEM + (ROPE ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
+  auto kern = attn_sk_kernel<BITS, ROPE, SCHED>;
+  const uint32_t smem = C::SMEM + (SCHED ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
   if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
@@ -442,7 +441,8 @@ cudaError_t launch_sk(const AttnArgs& a, cudaStream_t stream) {
 
 template <int BITS>
 cudaError_t launch_sk_bits(const AttnArgs& a, cudaStream_t s) {
-  return has_rope(a) ? launch_sk<BITS, true>(a, s) : launch_sk<BITS, false>(a, s);
+  if (!has_rope(a)) return launch_sk<BITS, false>(a, s);
+  return a.rope_mode == 2 ? launch_sk<BITS, true, true>(a, s) : launch_sk<BITS, true>(a, s);
 }
 
 }  // namespace

@@ -107,7 +107,7 @@ struct Cfg {
 
 }  // namespace
 
-template <int BITS, int D, int NQ, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE, bool SCHED>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnArgs a) {
   using C = Cfg<BITS, D, NQ>;
   constexpr int CPW = C::CPW;
@@ -170,9 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                               a.n_cached_blocks, bars);
   // rotary mode 2: the CTA's table of the 3D schedule, after the barrier region
   float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
-  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * C::NKV) / a.rope_frame : 0;
-  if constexpr (ROPE)
-    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kThreads);
+  const int rope_f0 = SCHED ? (tile0 * C::NKV) / a.rope_frame : 0;
+  if constexpr (SCHED) rope_table_build(a, rope_tab, rope_f0, kThreads);
   // query tiles -> K-major swizzled smem (rows past lq are zero).  The CH
   // chunks of a row are consecutive lanes of one warp in one pass, so with
   // fp16 operands they agree on the row's exponent by shuffles.
@@ -270,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp >= kDequantWarp0 || (NQ == 1 && warp >= 4)) {
     // ------------------------------------------------------------- dequant
     const int dt = warp >= kDequantWarp0 ? tid - kDequantWarp0 * 32 : kDequantThreads + tid - 128;
-    dequant_loop<C, BITS, D, ROPE>(a, bars, smem, sm_bs, dt, b, h, tile0, ntiles, kexp, rope_tab, rope_f0);
+    dequant_loop<C, BITS, D, ROPE, SCHED>(a, bars, smem, sm_bs, dt, b, h, tile0, ntiles, kexp, rope_tab, rope_f0);
   } else if ((warp >> 2) < NQ) {
     // ------------------------------------------------------------- softmax
     const int i = warp >> 2, r = (warp & 3) * 32 + lane;
@@ -293,14 +292,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
 namespace {
 
-template <int BITS, int D, int NQ, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE, bool SCHED = false>
 cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<BITS, D, NQ>;
-  auto kern = attn_tc_kernel<BITS, D, NQ, ROPE>;
+  auto kern = attn_tc_kernel<BITS, D, NQ, ROPE, SCHED>;
   // every CTA allocates all 512 TMEM columns: ask for enough shared memory
   // that no second CTA is placed on the SM to wait for them (plus the rotary
   // table of rope mode 2, which must fit)
-  const uint32_t extra = ROPE ? rope_table_bytes(a) : 0u;
+  const uint32_t extra = SCHED ? rope_table_bytes(a) : 0u;
   if (C::SMEM + extra > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   const uint32_t smem = std::max<uint32_t>(C::SMEM + extra, kSmemUsable / 2 + 1024);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -326,7 +325,8 @@ template <int BITS, int D>
 cudaError_t launch_d(const AttnArgs& a, cudaStream_t s) {
   if (has_rope(a)) {
     if constexpr (D == 64) {
-      if (a.kv_split) return launch_tc<BITS, D, 1, true>(a, s);
+      if (a.kv_split)
+        return a.rope_mode == 2 ? launch_tc<BITS, D, 1, true, true>(a, s) : launch_tc<BITS, D, 1, true>(a, s);
     }
     return cudaErrorInvalidConfiguration;
   }

@@ -92,7 +92,7 @@ constexpr int kThreads2 = kThreads + 32;
 
 }  // namespace
 
-template <int BITS, int D, int NQ, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE, bool SCHED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     attn_tc2_kernel(const __grid_constant__ AttnArgs a) {
   using C = Cfg2<BITS, D, NQ>;
@@ -159,9 +159,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   // rotary mode 2: the CTA's table of the 3D schedule, after the barrier
   // region (both CTAs of the pair cover the same tiles)
   float2* rope_tab = reinterpret_cast<float2*>(smem + C::OFF_BAR + kBarBytes);
-  const int rope_f0 = (ROPE && a.rope_mode == 2) ? (tile0 * C::NKV) / a.rope_frame : 0;
-  if constexpr (ROPE)
-    if (a.rope_mode == 2) rope_table_build(a, rope_tab, rope_f0, kThreads2);
+  const int rope_f0 = SCHED ? (tile0 * C::NKV) / a.rope_frame : 0;
+  if constexpr (SCHED) rope_table_build(a, rope_tab, rope_f0, kThreads2);
   // query tiles -> K-major swizzled smem (rows past lq are zero).  The CH
   // chunks of a row are consecutive lanes of one warp in one pass, so with
   // fp16 operands they agree on the row's exponent by shuffles.
@@ -318,7 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     // (row dv of the V tile = channel rank D/2 + dv, groups from partv)
     const int dt = tid - kDequantWarp0 * 32;
     const int dk = dt % D, partk = dt / D;
-    const RopeTable rtab = rope_table_of(a, rope_tab, dk, rope_f0);  // rotary mode 2 (keys only)
+    RopeTable rtab{};  // rotary mode 2 (keys only)
+    if constexpr (SCHED) rtab = rope_table_of(a, rope_tab, dk, rope_f0);
     const int dv = dt % C::DH, partv = dt / C::DH;
     const int64_t bh = int64_t(b) * a.heads + h;
     const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + dk;
@@ -419,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               x[jt] = v;
             }
           }
-          if (ROPE && tensor == 0) rope_rotate<C::GT, D>(a, rtab, x, tg, d);
+          if (ROPE && tensor == 0) rope_rotate<C::GT, D, SCHED>(a, rtab, x, tg, d);
 #pragma unroll
           for (int c = 0; c < C::GC; ++c) {
             uint32_t pk[4];
@@ -636,11 +636,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 
 namespace {
 
-template <int BITS, int D, int NQ, bool ROPE>
+template <int BITS, int D, int NQ, bool ROPE, bool SCHED = false>
 cudaError_t launch_tc2(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg2<BITS, D, NQ>;
-  auto kern = attn_tc2_kernel<BITS, D, NQ, ROPE>;
-  const uint32_t smem = C::SMEM + (ROPE ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
+  auto kern = attn_tc2_kernel<BITS, D, NQ, ROPE, SCHED>;
+  const uint32_t smem = C::SMEM + (SCHED ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
   if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
@@ -662,8 +662,13 @@ bool pair_two_tiles(const AttnArgs& a) {
 template <int BITS, int D>
 cudaError_t launch_d2(const AttnArgs& a, cudaStream_t s) {
   const bool rope = has_rope(a);
-  if (pair_two_tiles(a)) return rope ? launch_tc2<BITS, D, 2, true>(a, s) : launch_tc2<BITS, D, 2, false>(a, s);
-  return rope ? launch_tc2<BITS, D, 1, true>(a, s) : launch_tc2<BITS, D, 1, false>(a, s);
+  const bool sched = a.rope_mode == 2;
+  if (pair_two_tiles(a)) {
+    if (!rope) return launch_tc2<BITS, D, 2, false>(a, s);
+    return sched ? launch_tc2<BITS, D, 2, true, true>(a, s) : launch_tc2<BITS, D, 2, true>(a, s);
+  }
+  if (!rope) return launch_tc2<BITS, D, 1, false>(a, s);
+  return sched ? launch_tc2<BITS, D, 1, true, true>(a, s) : launch_tc2<BITS, D, 1, true>(a, s);
 }
 
 template <int BITS>

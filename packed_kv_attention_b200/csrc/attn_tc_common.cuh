@@ -460,28 +460,30 @@ __device__ __forceinline__ RopeTable rope_table_of(const AttnArgs& a, const floa
 // Pre-RoPE key mode: rotate pair (2i, 2i+1) of the GT dequantized values of
 // channel d, tokens tg .. tg + GT - 1, after rounding them to bf16 (the value
 // the cache would hold); the partner channel lives in the neighbour lane.
-// Rotation angles come from the caller's [T][D/2] tables (mode 1) or from the
-// CTA's table of the 3D schedule (mode 2).  Values past the attended tokens
-// are zero and stay zero.  tg is the same in every lane of the warp.
+// Values past the attended tokens are zero and stay zero.  tg is the same in
+// every lane of the warp.  (cos, sin) from the caller's [T][D/2] tables:
 template <int GT, int D>
-__device__ __forceinline__ void rope_rotate(const AttnArgs& a, const RopeTable& r, float (&x)[GT], int tg, int d) {
+__device__ __forceinline__ void rope_rotate_tables(const AttnArgs& a, float (&x)[GT], int tg, int d) {
   const int t_att = a.t_att;
-  if (a.rope_mode != 2) {
 #pragma unroll
-    for (int jt = 0; jt < GT; ++jt) {
-      const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
-      const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
-      const int t = tg + jt;
-      float c = 1.0f, s = 0.0f;
-      if (t < t_att) {
-        c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
-        s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
-      }
-      x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
+  for (int jt = 0; jt < GT; ++jt) {
+    const float xr = __bfloat162float(__float2bfloat16_rn(x[jt]));
+    const float other = __shfl_xor_sync(0xFFFFFFFFu, xr, 1);
+    const int t = tg + jt;
+    float c = 1.0f, s = 0.0f;
+    if (t < t_att) {
+      c = __ldg(a.rope_cos + int64_t(t) * (D / 2) + (d >> 1));
+      s = __ldg(a.rope_sin + int64_t(t) * (D / 2) + (d >> 1));
     }
-    return;
+    x[jt] = (d & 1) ? __fmaf_rn(other, s, xr * c) : __fmaf_rn(-other, s, xr * c);
   }
-  if (tg >= t_att) return;
+}
+
+// ... or from the CTA's table of the 3D schedule (rotary mode 2).
+template <int GT>
+__device__ __forceinline__ void rope_rotate_schedule(const AttnArgs& a, const RopeTable& r, float (&x)[GT], int tg,
+                                                     int d) {
+  if (tg >= a.t_att) return;
   const int f = div_magic_dev(tg, a.rope_frame_mul, a.rope_frame_shift);
   const int p = tg - f * a.rope_frame;
   const int row = div_magic_dev(p, a.rope_gw_mul, a.rope_gw_shift);
@@ -533,6 +535,14 @@ __device__ __forceinline__ void rope_rotate(const AttnArgs& a, const RopeTable& 
   }
 }
 
+template <int GT, int D, bool SCHED>
+__device__ __forceinline__ void rope_rotate(const AttnArgs& a, const RopeTable& r, float (&x)[GT], int tg, int d) {
+  if constexpr (SCHED)
+    rope_rotate_schedule<GT>(a, r, x, tg, d);
+  else
+    rope_rotate_tables<GT, D>(a, x, tg, d);
+}
+
 // The dequant warps of the single-CTA tensor-core kernels.  Thread dt owns
 // channel d = dt % D and the dequant groups part, part + TPC, ... of every KV
 // tile (a group = GT tokens = whole packed words and whole 16-byte chunks).
@@ -551,7 +561,7 @@ __device__ __forceinline__ void rope_rotate(const AttnArgs& a, const RopeTable& 
 // C provides CPW, GT, GW, GC, CPC, NKV, NG, TPC, PST, KST, VST, OFF_STAGE,
 // STAGE_BYTES, WORDS_BYTES, OFF_K, OFF_V, KV_BYTES and DEQ (the number of
 // dequant threads, the arrival count of kready/vready/empty).
-template <class C, int BITS, int D, bool ROPE>
+template <class C, int BITS, int D, bool ROPE, bool SCHED>
 __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, uint8_t* smem, const int* sm_bs, int dt,
                                              int b, int h, int tile0, int ntiles, int kexp, const float2* rope_tab,
                                              int rope_f0) {
@@ -567,7 +577,8 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
   const uint32_t* mgk = a.k_meta + bh * a.n_blocks_total * D + d;
   const uint32_t* mgv = a.v_meta + bh * a.n_blocks_total * D + d;
   const int nblk = a.n_cached_blocks;
-  const RopeTable rtab = rope_table_of(a, rope_tab, d, rope_f0);  // rotary mode 2
+  RopeTable rtab{};
+  if constexpr (SCHED) rtab = rope_table_of(a, rope_tab, d, rope_f0);
   // (scale, min) words of this thread's channel for block blk and blk + 1,
   // K and V, loaded one block ahead so a tile never waits on them
   uint32_t mk_cur = __ldg(mgk), mv_cur = __ldg(mgv);
@@ -664,7 +675,7 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
             x[jt] = v;
           }
         }
-        if (ROPE && tensor == 0) rope_rotate<C::GT, D>(a, rtab, x, tg, d);
+        if (ROPE && tensor == 0) rope_rotate<C::GT, D, SCHED>(a, rtab, x, tg, d);
 #pragma unroll
         for (int c = 0; c < C::GC; ++c) {
           uint32_t pk[4];
