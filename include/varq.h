@@ -352,6 +352,16 @@ VARQ_API const char* varq_status_string(int status);
 /* Library ABI version (incremented when a signature changes). */
 VARQ_API int varq_abi_version(void);
 
+/* Limit, in nanoseconds, of one internal pipeline wait of the tensor-core
+ * attention kernels (packed and dense) launched after this call returns,
+ * process-wide; 0 restores the default of 2 s.  Legitimate waits last
+ * microseconds; a wait that runs out makes the CTA stop, wait (up to 2 s)
+ * for the copies and MMAs it has already issued, free its tensor memory and
+ * return with VARQ_DEV_TIMEOUT set in dev_status.  That call's outputs are
+ * undefined; the context stays usable.  Meant for tests and for bounding a
+ * stalled launch.  Atomic; always returns VARQ_OK. */
+VARQ_API int varq_set_wait_limit_ns(uint64_t ns);
+
 #ifdef __cplusplus
 }
 #endif

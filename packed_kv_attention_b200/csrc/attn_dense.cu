@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(DenseCfg<D, NQ>::THREADS, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(DenseCfg<D, NQ>::THREADS, 1)
       mbar_init(&bars->vfree[s], 1);
     }
     mbar_init(&bars->teardown, 1);
-    bars->abort_flag = 0;
+    wait_ctl_init(&bars->ctl, a.wait_limit_ns);
     mbar_fence_init();
   }
   if (warp == C::MMA_WARP) {
@@ -125,14 +125,14 @@ __global__ void __launch_bounds__(DenseCfg<D, NQ>::THREADS, 1)
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % C::ST;
         const int tok0 = (tile0 + j) * NKV;
-        if (j >= C::ST && !mbar_wait(&bars->kfree[s], ((j / C::ST) - 1) & 1, abort_flag)) break;
+        if (j >= C::ST && !mbar_wait(&bars->kfree[s], ((j / C::ST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(&bars->kready[s], C::KV_BYTES);
 #pragma unroll
         for (int p = 0; p < D / 64; ++p)
           tma_load_4d(smem + C::OFF_K + s * C::KV_BYTES + p * C::PANEL_BYTES, &tm_k, p * 64, tok0, h, b,
                       &bars->kready[s]);
         nk = j + 1;
-        if (j >= C::ST && !mbar_wait(&bars->vfree[s], ((j / C::ST) - 1) & 1, abort_flag)) break;
+        if (j >= C::ST && !mbar_wait(&bars->vfree[s], ((j / C::ST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(&bars->vready[s], C::KV_BYTES);
 #pragma unroll
         for (int p = 0; p < D / 64; ++p)
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(DenseCfg<D, NQ>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  if (tid == 0 && bars->abort_flag) report(a.dev_status, VARQ_DEV_TIMEOUT);
+  if (tid == 0 && bars->ctl.abort) report(a.dev_status, VARQ_DEV_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ launch

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
   int* sm_bs = reinterpret_cast<int*>(smem + C::OFF_BAR + kBsOffset);
   int8_t* sm_qexp = reinterpret_cast<int8_t*>(smem + C::OFF_BAR + kQexpOffset);
   uint32_t* sm_tmax = reinterpret_cast<uint32_t*>(smem + C::OFF_TMAX);  // [4 warps][16 queries]
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
       mbar_init(&bars->sync2[i], 128);
     }
     mbar_init(&bars->teardown, 1);
-    bars->abort_flag = 0;
+    wait_ctl_init(&bars->ctl, a.wait_limit_ns);
     mbar_fence_init();
   }
   for (int i = tid; i <= a.n_cached_blocks; i += kSkThreads) sm_bs[i] = a.block_start[i];
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % C::PST;
-        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, abort_flag)) break;
+        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, ctl)) break;
         const int w0 = (tile0 + j) * C::NW;
         const int nw = min(C::NW, words_att - w0);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     int n_resc = 0;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      ok = wait_all(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag);
+      ok = wait_all(&bars->s_full[j & 1], (j >> 1) & 1, ctl);
       if (!ok) break;
       tc_fence_after();
       // y = s sl2 - m (the exp2 argument against the running maximum), in
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
       const bool exceed = __any_sync(0xFFFFFFFFu, ymax > kRescaleThreshold);
       if (lane == 0) bars->flag[j & 1][warp] = exceed ? 1u : 0u;
       mbar_arrive(&bars->sync[j & 1]);
-      ok = wait_all(&bars->sync[j & 1], (j >> 1) & 1, abort_flag);
+      ok = wait_all(&bars->sync[j & 1], (j >> 1) & 1, ctl);
       if (!ok) break;
       const volatile uint32_t* fl = bars->flag[j & 1];
       if ((fl[0] | fl[1] | fl[2] | fl[3]) != 0u) {
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
           if (lane == i) sm_tmax[warp * kSkN + i] = u;
         }
         mbar_arrive(&bars->sync2[n_resc & 1]);
-        ok = wait_all(&bars->sync2[n_resc & 1], (n_resc >> 1) & 1, abort_flag);
+        ok = wait_all(&bars->sync2[n_resc & 1], (n_resc >> 1) & 1, ctl);
         ++n_resc;
         if (!ok) break;
         // O^T holds the earlier tiles once P V(j - 1) has finished (P V(j - 2)
@@ -325,10 +325,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
         uint32_t o[kSkN];
         if (j >= 1) {
           if (j >= 2) {
-            ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag);
+            ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, ctl);
             if (!ok) break;
           }
-          ok = wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag);
+          ok = wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl);
           if (!ok) break;
           tc_fence_after();
           tmem_ld16(lane_base + 2u * kSkN, o);
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
       }
       // P buffer j & 1 is free once P V(j - 2) has finished
       if (j >= 2) {
-        ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag);
+        ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, ctl);
         if (!ok) break;
       }
       uint8_t* pb = smem + C::OFF_P + (j & 1) * C::P_BYTES + p_thread;
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     // ------------------------------------------------------------- epilogue
     // O^T is final once P V of the last two tiles has finished
     bool have = ok && ntiles > 0;
-    if (have && ntiles >= 2) have = wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, abort_flag);
-    if (have) have = wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag);
+    if (have && ntiles >= 2) have = wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, ctl);
+    if (have) have = wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, ctl);
     // row sums: partial per token position -> per query over the 128 threads
 #pragma unroll
     for (int i = 0; i < kSkN; ++i) {
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     }
     const int je = ntiles;  // one more exchange, on the next tile parity's barrier
     mbar_arrive(&bars->sync[je & 1]);
-    if (have) have = wait_all(&bars->sync[je & 1], (je >> 1) & 1, abort_flag);
+    if (have) have = wait_all(&bars->sync[je & 1], (je >> 1) & 1, ctl);
     float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2);
     if (have) {
       tc_fence_after();
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) attn_sk_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem, kSkTmemCols);
   }
-  if (tid == 0 && bars->abort_flag) report(a.dev_status, VARQ_DEV_TIMEOUT);
+  if (tid == 0 && bars->ctl.abort) report(a.dev_status, VARQ_DEV_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ launch

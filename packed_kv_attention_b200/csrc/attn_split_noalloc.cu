@@ -86,6 +86,7 @@ extern "C" VARQ_API int varq_packed_attention_noalloc(
 
   varq::AttnArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.wait_limit_ns = varq::wait_limit_ns();
   a.words_per_row = L->words_per_row;
   a.batch = L->batch;
   a.heads = L->heads;

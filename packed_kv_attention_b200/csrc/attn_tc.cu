@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
   int* sm_bs = reinterpret_cast<int*>(smem + C::OFF_BAR + kBsOffset);  // block_start[0..n_cached_blocks]
   int8_t* sm_qexp = reinterpret_cast<int8_t*>(smem + C::OFF_BAR + kQexpOffset);  // pre-RoPE: per-row query exponents
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&bars->o_done[i], 1);
     }
     mbar_init(&bars->teardown, 1);
-    bars->abort_flag = 0;
+    wait_ctl_init(&bars->ctl, a.wait_limit_ns);
     mbar_fence_init();
   }
   for (int i = tid; i <= a.n_cached_blocks; i += kThreads) sm_bs[i] = a.block_start[i];
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % C::PST;
-        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, abort_flag)) break;
+        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, ctl)) break;
         const int w0 = (tile0 + j) * C::NW;
         const int nw = min(C::NW, words_att - w0);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  if (tid == 0 && bars->abort_flag) report(a.dev_status, VARQ_DEV_TIMEOUT);
+  if (tid == 0 && bars->ctl.abort) report(a.dev_status, VARQ_DEV_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ launch

@@ -110,7 +110,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
   int* sm_bs = reinterpret_cast<int*>(smem + C::OFF_BAR + kBsOffset);  // block_start[0..n_cached_blocks]
   int8_t* sm_qexp = reinterpret_cast<int8_t*>(smem + C::OFF_BAR + kQexpOffset);  // pre-RoPE: per-row query exponents
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -143,7 +143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       mbar_init(&bars->o_done[i], 1);
     }
     mbar_init(&bars->teardown, 1);
-    bars->abort_flag = 0;
+    wait_ctl_init(&bars->ctl, a.wait_limit_ns);
     mbar_fence_init();
   }
   for (int i = tid; i <= a.n_cached_blocks; i += kThreads2) sm_bs[i] = a.block_start[i];
@@ -205,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % C::PST;
-        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, abort_flag)) break;
+        if (j >= C::PST && !mbar_wait(&bars->empty[st], ((j / C::PST) & 1) ^ 1, ctl)) break;
         const int w0 = (tile0 + j) * C::NW;
         const int nw = min(C::NW, words_att - w0);
         uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
@@ -255,7 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           mma2_ts(tmem + col_o<NQ>(i), tmem + col_s(i) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = ntiles > 0 && mbar_wait_cluster(&bars->kready[0], 0, abort_flag);
+      bool ok = ntiles > 0 && mbar_wait_cluster(&bars->kready[0], 0, ctl);
       if (ok) {
         tc_fence_after();
         for (int i = 0; i < NQ; ++i) {
@@ -265,9 +265,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         mma2_commit_both(&bars->kfree[0]);
       }
       for (int j = 0; j < ntiles && ok; ++j) {
-        ok = mbar_wait_cluster(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag);
+        ok = mbar_wait_cluster(&bars->vready[j % C::VST], (j / C::VST) & 1, ctl);
         for (int i = 0; i < NQ && ok; ++i) {
-          ok = mbar_wait_cluster(&bars->p_ready[i], j & 1, abort_flag);
+          ok = mbar_wait_cluster(&bars->p_ready[i], j & 1, ctl);
           if (!ok) break;
           tc_fence_after();
           issue_pv(i, j);
@@ -275,7 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           if (i == NQ - 1) mma2_commit_both(&bars->vfree[j % C::VST]);
           if (j + 1 < ntiles) {
             if (i == 0) {
-              ok = mbar_wait_cluster(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, abort_flag);
+              ok = mbar_wait_cluster(&bars->kready[(j + 1) % C::KST], ((j + 1) / C::KST) & 1, ctl);
               if (!ok) break;
               tc_fence_after();
             }
@@ -295,7 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j)
         for (int i = 0; i < NQ && ok; ++i) {
-          ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
+          ok = mbar_wait(&bars->p_ready[i], j & 1, ctl);
           if (ok) mbar_arrive_rank(&bars->p_ready[i], 0);
         }
       mbar_wait_drain(&bars->teardown, 0);
@@ -304,9 +304,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     // ------------------------------------------------------------- relay
     if (rank == 1 && lane == 0) {
       for (int j = 0; j < ntiles; ++j) {
-        if (!mbar_wait(&bars->kready[j % C::KST], (j / C::KST) & 1, abort_flag)) break;
+        if (!mbar_wait(&bars->kready[j % C::KST], (j / C::KST) & 1, ctl)) break;
         mbar_arrive_rank(&bars->kready[j % C::KST], 0);
-        if (!mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, abort_flag)) break;
+        if (!mbar_wait(&bars->vready[j % C::VST], (j / C::VST) & 1, ctl)) break;
         mbar_arrive_rank(&bars->vready[j % C::VST], 0);
       }
     }
@@ -341,14 +341,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         mv_next = more ? __ldg(mgv + int64_t(blk + 1) * D) : 0u;
       }
       const int blk_lo = blk;
-      if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
+      if (!wait_all(&bars->full[st], (j / C::PST) & 1, ctl)) break;
       const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
       bool ok = true;
       for (int tensor = 0; tensor < 2 && ok; ++tensor) {
         const int nbuf = tensor == 0 ? C::KST : C::VST;
         const int buf = j % nbuf;
         uint64_t* freeb = tensor == 0 ? &bars->kfree[buf] : &bars->vfree[buf];
-        if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, abort_flag)) {
+        if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, ctl)) {
           ok = false;
           break;
         }
@@ -435,7 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         fence_async_smem();
         mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
       }
-      if (!ok || *abort_flag) break;
+      if (!ok || ctl->abort) break;
       mbar_arrive(&bars->empty[st]);
     }
   } else if ((warp >> 2) < NQ) {
@@ -451,7 +451,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      ok = wait_all(&bars->s_full[i], j & 1, abort_flag);
+      ok = wait_all(&bars->s_full[i], j & 1, ctl);
       if (!ok) break;
       tc_fence_after();
       const int valid = min(C::NKV, t_att - (tile0 + j) * C::NKV);
@@ -491,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       const float alpha = (j == 0) ? 0.0f : ex2_approx(m_run - m_new);
       // PV_i of the previous tile has finished before O_i is rescaled
       if (j >= 1) {
-        ok = wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
+        ok = wait_all(&bars->o_done[i], (j - 1) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xFFFFFFFFu, m_new != m_run)) {
@@ -575,7 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       const int row = qblk * (NQ * BM) + i * BM + r;
       float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
                   int64_t(row) * (D + 2);
-      const bool have = ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
+      const bool have = ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, ctl);
       if (have) {
         tc_fence_after();
 #pragma unroll 1
@@ -595,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         ws[D] = have ? m_run : -__int_as_float(0x7F800000);
         ws[D + 1] = have ? l_run : 0.0f;
       }
-    } else if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag)) {
+    } else if (ok && ntiles > 0 && wait_all(&bars->o_done[i], (ntiles - 1) & 1, ctl)) {
       tc_fence_after();
       const int row = qblk * (NQ * BM) + i * BM + r;
       const float inv = 1.0f / l_run;
@@ -629,7 +629,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     tc_fence_after();
     tmem2_dealloc(tmem, C::TMEM_COLS);
   }
-  if (tid == 0 && bars->abort_flag) report(a.dev_status, VARQ_DEV_TIMEOUT);
+  if (tid == 0 && bars->ctl.abort) report(a.dev_status, VARQ_DEV_TIMEOUT);
 }
 
 // ------------------------------------------------------------------ launch

@@ -37,7 +37,7 @@ struct Barriers {
   uint64_t o_done[2];             // PV_i finished
   uint64_t teardown;
   uint32_t tmem_base;
-  int abort_flag;
+  WaitCtl ctl;                    // abort flag and wait limit
   uint32_t kmax[24];              // pre-RoPE keys: per-warp largest |min| + (2^b - 1) scale
   alignas(16) uint32_t flag[2][4];  // swap-AB split kernel: per-warp softmax votes, by tile parity
   uint64_t sync[2], sync2[2];     // swap-AB split kernel: softmax-warp exchanges, by tile parity
@@ -75,8 +75,8 @@ __device__ __forceinline__ int rope_key_exponent_of(const Barriers* bars) {
   return rope_key_exponent(mb);
 }
 
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile WaitCtl* ctl) {
+  const bool ok = mbar_wait(bar, parity, ctl);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
@@ -102,14 +102,14 @@ __device__ __forceinline__ uint32_t o_col_of(int i) {
 // kfree/vfree by commits once the MMAs reading them have finished.
 template <int NQ, bool DB, int KST, int VST, class QK, class PV>
 __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& issue_qk, PV&& issue_pv) {
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
   if constexpr (DB) {
     // one query tile: S(0), S(1) first, then per KV tile j PV(j) and S(j + 2)
     // into the buffer P(j) is read from (the MMAs run in issue order);
     // barriers indexed by j & 1
     bool ok = true;
     for (int j = 0; j < min(2, ntiles) && ok; ++j) {
-      ok = mbar_wait(&bars->kready[j % KST], (j / KST) & 1, abort_flag);
+      ok = mbar_wait(&bars->kready[j % KST], (j / KST) & 1, ctl);
       if (!ok) break;
       tc_fence_after();
       issue_qk(0, j);
@@ -117,15 +117,15 @@ __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& 
       mma_commit(&bars->kfree[j % KST]);
     }
     for (int j = 0; j < ntiles && ok; ++j) {
-      ok = mbar_wait(&bars->vready[j % VST], (j / VST) & 1, abort_flag) &&
-           mbar_wait(&bars->p_ready[j & 1], (j >> 1) & 1, abort_flag);
+      ok = mbar_wait(&bars->vready[j % VST], (j / VST) & 1, ctl) &&
+           mbar_wait(&bars->p_ready[j & 1], (j >> 1) & 1, ctl);
       if (!ok) break;
       tc_fence_after();
       issue_pv(0, j);
       mma_commit(&bars->o_done[j & 1]);
       mma_commit(&bars->vfree[j % VST]);
       if (j + 2 < ntiles) {
-        ok = mbar_wait(&bars->kready[(j + 2) % KST], ((j + 2) / KST) & 1, abort_flag);
+        ok = mbar_wait(&bars->kready[(j + 2) % KST], ((j + 2) / KST) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         issue_qk(0, j + 2);
@@ -134,7 +134,7 @@ __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& 
       }
     }
   } else {
-    bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, abort_flag);
+    bool ok = ntiles > 0 && mbar_wait(&bars->kready[0], 0, ctl);
     if (ok) {
       tc_fence_after();
       for (int i = 0; i < NQ; ++i) {
@@ -144,9 +144,9 @@ __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& 
       mma_commit(&bars->kfree[0]);
     }
     for (int j = 0; j < ntiles && ok; ++j) {
-      ok = mbar_wait(&bars->vready[j % VST], (j / VST) & 1, abort_flag);
+      ok = mbar_wait(&bars->vready[j % VST], (j / VST) & 1, ctl);
       for (int i = 0; i < NQ && ok; ++i) {
-        ok = mbar_wait(&bars->p_ready[i], j & 1, abort_flag);
+        ok = mbar_wait(&bars->p_ready[i], j & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         issue_pv(i, j);
@@ -154,7 +154,7 @@ __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& 
         if (i == NQ - 1) mma_commit(&bars->vfree[j % VST]);
         if (j + 1 < ntiles) {
           if (i == 0) {
-            ok = mbar_wait(&bars->kready[(j + 1) % KST], ((j + 1) / KST) & 1, abort_flag);
+            ok = mbar_wait(&bars->kready[(j + 1) % KST], ((j + 1) / KST) & 1, ctl);
             if (!ok) break;
             tc_fence_after();
           }
@@ -181,7 +181,7 @@ __device__ __forceinline__ void mma_issue_loop(Barriers* bars, int ntiles, QK&& 
 template <int NKV, int D, int NQ, bool DB>
 __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, uint32_t tmem, int warp, int lane,
                                              int qblk, int split, int b, int h, int tile0, int ntiles, float sl2) {
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
   const int t_att = a.t_att;
   const int i = warp >> 2;                 // query tile of this warpgroup
   const int r = (warp & 3) * 32 + lane;    // row within the tile == TMEM lane
@@ -193,8 +193,8 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
   for (int j = 0; j < ntiles && ok; ++j) {
     // S of this tile: TMEM columns and barrier (buffer j & 1 when double-buffered)
     const uint32_t s_tmem = lane_base + s_col_of<NQ, DB>(i, j);
-    ok = DB ? wait_all(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag)
-               : wait_all(&bars->s_full[i], j & 1, abort_flag);
+    ok = DB ? wait_all(&bars->s_full[j & 1], (j >> 1) & 1, ctl)
+               : wait_all(&bars->s_full[i], j & 1, ctl);
     if (!ok) break;
     tc_fence_after();
     const int valid = min(NKV, t_att - (tile0 + j) * NKV);
@@ -238,12 +238,12 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
     // waited for and PV(t + 2) cannot have run: PV(j - 2) is waited for every
     // tile (long finished), PV(j - 1) only to rescale O.
     if (DB && j >= 2) {
-      ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag);
+      ok = wait_all(&bars->o_done[j & 1], ((j - 2) >> 1) & 1, ctl);
       if (!ok) break;
     }
     if (j >= 1 && (!DB || __any_sync(0xFFFFFFFFu, m_new != m_run))) {
-      ok = DB ? wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)
-                 : wait_all(&bars->o_done[i], (j - 1) & 1, abort_flag);
+      ok = DB ? wait_all(&bars->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl)
+                 : wait_all(&bars->o_done[i], (j - 1) & 1, ctl);
       if (!ok) break;
       tc_fence_after();
       if (__any_sync(0xFFFFFFFFu, m_new != m_run)) {
@@ -325,10 +325,10 @@ __device__ __forceinline__ void softmax_loop(const AttnArgs& a, Barriers* bars, 
   // the last two tiles, waited for in order)
   auto o_final = [&]() {
     if constexpr (DB) {
-      return (ntiles < 2 || wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, abort_flag)) &&
-             wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag);
+      return (ntiles < 2 || wait_all(&bars->o_done[ntiles & 1], ((ntiles - 2) >> 1) & 1, ctl)) &&
+             wait_all(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, ctl);
     } else {
-      return wait_all(&bars->o_done[i], (ntiles - 1) & 1, abort_flag);
+      return wait_all(&bars->o_done[i], (ntiles - 1) & 1, ctl);
     }
   };
   if (a.kv_split) {
@@ -569,7 +569,7 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   constexpr bool QK_F16 = ROPE;
   static_assert(C::GT == dequant_group_tokens(BITS), "rotary table rows assume the host's group size");
-  volatile int* abort_flag = &bars->abort_flag;
+  volatile WaitCtl* ctl = &bars->ctl;
   const int t_att = a.t_att;
   const int d = dt % D;
   const int part = dt / D;
@@ -596,14 +596,14 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
       mv_next = more ? __ldg(mgv + int64_t(blk + 1) * D) : 0u;
     }
     const int blk_lo = blk;
-    if (!wait_all(&bars->full[st], (j / C::PST) & 1, abort_flag)) break;
+    if (!wait_all(&bars->full[st], (j / C::PST) & 1, ctl)) break;
     const uint8_t* sb = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
     bool ok = true;
     for (int tensor = 0; tensor < 2 && ok; ++tensor) {
       const int nbuf = tensor == 0 ? C::KST : C::VST;
       const int buf = j % nbuf;
       uint64_t* freeb = tensor == 0 ? &bars->kfree[buf] : &bars->vfree[buf];
-      if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, abort_flag)) {
+      if (j >= nbuf && !wait_all(freeb, ((j / nbuf) - 1) & 1, ctl)) {
         ok = false;
         break;
       }
@@ -691,7 +691,7 @@ __device__ __forceinline__ void dequant_loop(const AttnArgs& a, Barriers* bars, 
       fence_async_smem();
       mbar_arrive(tensor == 0 ? &bars->kready[buf] : &bars->vready[buf]);
     }
-    if (!ok || *abort_flag) break;
+    if (!ok || ctl->abort) break;
     mbar_arrive(&bars->empty[st]);
   }
 }

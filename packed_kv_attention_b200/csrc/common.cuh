@@ -36,7 +36,8 @@ __device__ __forceinline__ void report(uint32_t* dev_status, uint32_t bits) {
   if (dev_status != nullptr) atomicOr(dev_status, bits);
 }
 
-// Wall-clock limit of one barrier wait.  Legitimate waits last microseconds.
+// Default wall-clock limit of one barrier wait.  Legitimate waits last
+// microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ------------------------------------------------------------- mbarriers
@@ -84,20 +85,38 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar_addr, uint32_
   return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed.  Returns false
-// (and flags *abort) when the limit runs out or another thread aborted.  The
-// waiting thread sleeps inside try_wait, so spinning warps do not take issue
-// slots from the warps that do the work.
+// Pipeline control word of one CTA, in shared memory: the abort flag (set by
+// the first wait that runs out; every later wait then gives up at once) and
+// this launch's wait limit.
 constexpr uint32_t kSuspendHintNs = 200000;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+struct WaitCtl {
+  int abort;
+  uint32_t hint_ns;   // suspend hint of one try_wait: min(kSuspendHintNs, limit_ns)
+  uint64_t limit_ns;  // wall-clock limit of one wait
+};
+// limit_ns == 0 selects kWaitLimitNs (one thread, before the set-up barrier).
+__device__ __forceinline__ void wait_ctl_init(WaitCtl* c, uint64_t limit_ns) {
+  const uint64_t l = limit_ns == 0 ? kWaitLimitNs : limit_ns;
+  c->abort = 0;
+  c->limit_ns = l;
+  c->hint_ns = static_cast<uint32_t>(l < kSuspendHintNs ? l : kSuspendHintNs);
+}
+
+// Wait until the phase with the given parity has completed.  Returns false
+// (and sets ctl->abort) when the limit runs out or another thread aborted.
+// The waiting thread sleeps inside try_wait, so spinning warps do not take
+// issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile WaitCtl* ctl) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_suspend(a, parity, kSuspendHintNs)) return true;
+  const uint32_t hint = ctl->hint_ns;
+  if (mbar_try_wait_suspend(a, parity, hint)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = ctl->limit_ns;
   for (;;) {
-    if (mbar_try_wait_suspend(a, parity, kSuspendHintNs)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
+    if (mbar_try_wait_suspend(a, parity, hint)) return true;
+    if (ctl->abort) return false;
+    if (global_timer_ns() - t0 > limit) {
+      ctl->abort = 1;
       return false;
     }
   }
@@ -137,8 +156,9 @@ __device__ __forceinline__ void mbar_arrive_rank(uint64_t* bar, uint32_t rank) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 // mbar_wait with cluster-scope acquire (arrivals come from other CTAs).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile WaitCtl* ctl) {
   const uint32_t a = smem_u32(bar);
+  const uint32_t hint = ctl->hint_ns;
   auto try_wait = [&]() {
     uint32_t ok;
     asm volatile(
@@ -146,17 +166,18 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(a), "r"(parity), "r"(kSuspendHintNs)
+        : "r"(a), "r"(parity), "r"(hint)
         : "memory");
     return ok != 0;
   };
   if (try_wait()) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = ctl->limit_ns;
   for (;;) {
     if (try_wait()) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
+    if (ctl->abort) return false;
+    if (global_timer_ns() - t0 > limit) {
+      ctl->abort = 1;
       return false;
     }
   }

@@ -99,6 +99,7 @@ struct AttnArgs {
   int32_t kv_split;        // 1: each CTA attends to one of n_splits ranges of KV tiles and writes an
                            // unnormalised partial (O, m, l) to the workspace; a combine kernel merges them
   int32_t n_splits;
+  uint64_t wait_limit_ns;  // limit of one pipeline wait (0: the default, 2 s)
   // pre-RoPE key mode: 0 none, 1 caller tables (rope_cos, rope_sin), 2 a 3D
   // rotary schedule whose angles each CTA computes (frame, row, column axes)
   int32_t rope_mode;
@@ -122,6 +123,8 @@ struct DenseTensor {
 };
 
 inline bool has_rope(const AttnArgs& a) { return a.rope_mode != 0; }
+// The wait limit varq_set_wait_limit_ns last set (0: the default).
+uint64_t wait_limit_ns();
 // Tokens per KV tile of the packed-cache attention kernels for a bit width:
 // whole words of whole 16-token MMA slices, at most 128 (128, 96 for 5-bit, 80
 // for 3- and 6-bit).

@@ -1,6 +1,8 @@
 // Host side of the C ABI declared in include/varq.h: argument validation,
-// layout planning and kernel dispatch.  No allocation, no global state.
+// layout planning and kernel dispatch.  No allocation; the only global state
+// is the pipeline wait limit (an atomic).
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -18,11 +20,22 @@ using varq::stride_ok;
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? VARQ_OK : VARQ_ERR_CUDA; }
 
+std::atomic<uint64_t> g_wait_limit_ns{0};
+
 }  // namespace
+
+namespace varq {
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+}  // namespace varq
 
 extern "C" {
 
 int varq_abi_version(void) { return 1; }
+
+int varq_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return VARQ_OK;
+}
 
 const char* varq_status_string(int status) {
   switch (status) {
@@ -144,6 +157,7 @@ static int choose_path(int lq, int path) {
 
 static void fill_attn(AttnArgs& a, const varq_cache_layout* L, int lq, int n_cached_blocks) {
   std::memset(&a, 0, sizeof(a));
+  a.wait_limit_ns = varq::wait_limit_ns();
   a.words_per_row = L->words_per_row;
   a.batch = L->batch;
   a.heads = L->heads;
@@ -307,6 +321,7 @@ static int check_dense(int batch, int heads, int head_dim, int64_t n_tokens, int
 
 static void fill_dense(AttnArgs& a, int batch, int heads, int head_dim, int64_t n_tokens, int lq) {
   std::memset(&a, 0, sizeof(a));
+  a.wait_limit_ns = varq::wait_limit_ns();
   a.batch = batch;
   a.heads = heads;
   a.head_dim = head_dim;

@@ -21,6 +21,7 @@ __all__ = [
     "DEV_NONFINITE", "DEV_META_OVERFLOW", "DEV_TIMEOUT",
     "varq_packed_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "varq_quantize_pack_launches",
     "varq_dense_attention", "varq_dense_attention_workspace", "Rope3d", "varq_packed_attention_rope3d",
+    "varq_set_wait_limit_ns",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvarq.so")
@@ -112,6 +113,8 @@ def lib() -> ctypes.CDLL:
             _c_p, _c_p, _c_p, _c_p, _c_int, _c_f, ctypes.POINTER(Rope3d),
             _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_int, _c_p, _c_p]
         L.varq_packed_attention_rope3d.restype = _c_int
+        L.varq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.varq_set_wait_limit_ns.restype = _c_int
         L.varq_status_string.argtypes = [_c_int]
         L.varq_status_string.restype = ctypes.c_char_p
         L.varq_abi_version.argtypes = []
@@ -338,3 +341,9 @@ def varq_packed_attention_rope3d(layout: CacheLayout, q: torch.Tensor, k_packed:
         ctypes.byref(rope), _ptr(out), out.stride(0), out.stride(1), out.stride(2),
         _ptr(lse), _ptr(workspace), ws_bytes, path, _ptr(dev_status), _stream(stream))
     _check(rc, "varq_packed_attention_rope3d")
+
+
+def varq_set_wait_limit_ns(ns: int) -> None:
+    """Limit of one internal pipeline wait of later attention launches (0:
+    the default, 2 s).  A wait that runs out sets VARQ_DEV_TIMEOUT."""
+    _check(lib().varq_set_wait_limit_ns(int(ns)), "varq_set_wait_limit_ns")

@@ -217,6 +217,12 @@ def test_dense_attention_errors():
     assert V.varq_dense_attention_workspace(2, 4, 128, 4, 1000, V.PATH_TENSOR) == 0
 
 
+def test_wait_limit_knob():
+    lib = V.lib()
+    assert lib.varq_set_wait_limit_ns(5000) == OK
+    assert lib.varq_set_wait_limit_ns(0) == OK   # back to the default
+
+
 def test_status_strings():
     for c in (OK, INVALID, UNSUPPORTED, CUDA, WORKSPACE, ALIGN):
         assert V.varq_status_string(c).startswith("VARQ_")
