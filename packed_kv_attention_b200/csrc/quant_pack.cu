@@ -22,13 +22,16 @@
 //
 // Arithmetic is the exact fp32 definition:
 //   s = fp32(fp32(max - min) / (2^b - 1)),  q = rint(fp32(fp32(x - min) / s)).
-// Fast path: y = fma(x, fp32(1/s), -fp32(min/s)) and q = rint(y) via the
-// 1.5*2^23 rounding constant.  y differs from the correctly rounded quotient
-// by less than delta = 2^-21 (2|min/s| + 2^b + 2) (a few fp32 roundings of
-// terms bounded by |min/s| and 2^b), so wherever y lies farther than delta
-// from a half-integer both round to the same integer.  The fast path is
-// branch-free; a code inside that window (or with a non-finite y) is marked
-// and recomputed alone with __fdiv_rn afterwards.
+// The quotient is formed exactly without a division: with r = RN(1/s) per
+// cell, d = RN(x - min), q0 = RN(d r), the residual e = d - q0 s (exact in one
+// fma) and q1 = RN(q0 + e r), Markstein's theorem (correction step of a
+// quotient with a correctly rounded reciprocal; J.-M. Muller et al.,
+// "Handbook of Floating-Point Arithmetic", the FMA-based division section)
+// gives q1 = RN(d / s).  rint(q1) then comes from adding 1.5*2^23 (ties to
+// even, as rint): five operations a code, no branch.  Cells where the
+// theorem's range conditions may not hold -- non-finite constants, or s
+// below 2^-100 (so that e could fall below the subnormal grid) -- take
+// __fdiv_rn for every code.
 #include <algorithm>
 
 #include "common.cuh"
@@ -91,14 +94,12 @@ __device__ __forceinline__ Item decode(const QuantArgs& a, int64_t item) {
 
 struct Partial {
   __nv_bfloat162 mn2[4], mx2[4];
-  bool seen;
   __device__ __forceinline__ void init() {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       mn2[i] = as_bf2(0x7F807F80u);
       mx2[i] = as_bf2(0xFF80FF80u);
     }
-    seen = false;
   }
   __device__ __forceinline__ void add(const uint4& v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -107,89 +108,94 @@ struct Partial {
       mn2[i] = __hmin2_nan(mn2[i], as_bf2(w[i]));
       mx2[i] = __hmax2_nan(mx2[i], as_bf2(w[i]));
     }
-    seen = true;
   }
 };
 
 // Per-thread partials -> per-channel min/max of the block (threads tid < G
-// receive channel tid).  Returns whether any input was NaN or infinite.
+// receive channel tid).  The butterfly runs on packed bf16 pairs (exact:
+// min/max only select); a NaN or infinite input shows as a non-finite min or
+// max of its channel, which the caller reports.
 template <int G>
-__device__ __forceinline__ bool block_reduce(Partial& p, float (*red_mn)[G], float (*red_mx)[G], float& out_mn,
+__device__ __forceinline__ void block_reduce(Partial& p, float (*red_mn)[G], float (*red_mx)[G], float& out_mn,
                                              float& out_mx) {
   constexpr int TPR = G / 8;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c8 = (tid % TPR) * 8;
-  float mn[8], mx[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    mn[2 * i] = __low2float(p.mn2[i]);
-    mn[2 * i + 1] = __high2float(p.mn2[i]);
-    mx[2 * i] = __low2float(p.mx2[i]);
-    mx[2 * i + 1] = __high2float(p.mx2[i]);
-  }
-  // a NaN or infinite input shows in this thread's NaN-propagating min/max
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) bad |= p.seen && !(fabsf(mn[i]) <= 3.4e38f && fabsf(mx[i]) <= 3.4e38f);
   // lanes with equal tid % TPR hold the same channels: butterfly over the others
 #pragma unroll
   for (int off = TPR; off < 32; off <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      mn[i] = fminf(mn[i], __shfl_xor_sync(0xFFFFFFFFu, mn[i], off));
-      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xFFFFFFFFu, mx[i], off));
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t mn = __shfl_xor_sync(0xFFFFFFFFu, *reinterpret_cast<uint32_t*>(&p.mn2[i]), off);
+      const uint32_t mx = __shfl_xor_sync(0xFFFFFFFFu, *reinterpret_cast<uint32_t*>(&p.mx2[i]), off);
+      p.mn2[i] = __hmin2_nan(p.mn2[i], as_bf2(mn));
+      p.mx2[i] = __hmax2_nan(p.mx2[i], as_bf2(mx));
     }
   }
   if (lane < TPR) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      red_mn[warp][c8 + i] = mn[i];
-      red_mx[warp][c8 + i] = mx[i];
+    for (int i = 0; i < 4; ++i) {
+      red_mn[warp][c8 + 2 * i] = __low2float(p.mn2[i]);
+      red_mn[warp][c8 + 2 * i + 1] = __high2float(p.mn2[i]);
+      red_mx[warp][c8 + 2 * i] = __low2float(p.mx2[i]);
+      red_mx[warp][c8 + 2 * i + 1] = __high2float(p.mx2[i]);
     }
   }
-  const bool any_bad = __syncthreads_or(bad ? 1 : 0) != 0;
+  __syncthreads();
   if (tid < G) {
+    // NaN-propagating across warps as within them
     float m0 = red_mn[0][tid], m1 = red_mx[0][tid];
+    bool nan = m0 != m0 || m1 != m1;
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) {
-      m0 = fminf(m0, red_mn[w][tid]);
-      m1 = fmaxf(m1, red_mx[w][tid]);
+      const float a = red_mn[w][tid], b = red_mx[w][tid];
+      nan |= a != a || b != b;
+      m0 = fminf(m0, a);
+      m1 = fmaxf(m1, b);
     }
-    out_mn = m0;
-    out_mx = m1;
+    out_mn = nan ? __int_as_float(0x7FC00000) : m0;
+    out_mx = nan ? __int_as_float(0x7FC00000) : m1;
   }
-  return any_bad;
 }
 
 // Cell constants and the metadata word of channel tid (thread tid < G).
 template <int BITS, int G>
 __device__ __forceinline__ void cell_constants(const QuantArgs& a, const Item& it, float m0, float m1, float* cell_s,
-                                               float* cell_r, float* cell_nmr, float* cell_m, float* cell_dl) {
+                                               float* cell_r, float* cell_m, uint32_t* cell_fast) {
   constexpr float QMAX = float((1u << BITS) - 1u);
   const int tid = threadIdx.x;
   const float s = __fdiv_rn(__fsub_rn(m1, m0), QMAX);
   const float rcp = s == 0.0f ? 0.0f : __frcp_rn(s);
-  const float mr = __fmul_rn(m0, rcp);
   cell_s[tid] = s;
   cell_r[tid] = rcp;
-  cell_nmr[tid] = -mr;
   cell_m[tid] = m0;
-  cell_dl[tid] = 0.5f - (2.0f * fabsf(mr) + float(1u << BITS) + 2.0f) * 4.76837158203125e-7f;  // 0.5 - delta
+  // the division-free quotient's conditions (a constant cell, s == 0, gives
+  // d = 0 and code 0 through it as well)
+  const bool finite = fabsf(m0) <= 3.4e38f && fabsf(s) <= 3.4e38f && fabsf(rcp) <= 3.4e38f;
+  cell_fast[tid] = (finite && (s == 0.0f || s >= 7.888609052210118e-31f)) ? 1u : 0u;  // 2^-100
   const uint32_t lo = __half_as_ushort(__float2half_rn(s));
   const uint32_t hi = __half_as_ushort(__float2half_rn(m0));
   a.meta[((int64_t(it.b) * a.heads + it.h) * a.n_blocks_total + it.k) * a.head_dim + it.g * G + tid] = lo | (hi << 16);
   if (!(fabsf(m0) <= 65504.0f) || !(s <= 65504.0f)) report(a.dev_status, VARQ_DEV_META_OVERFLOW);
 }
 
+// The code of x in a cell as (1.5*2^23 + code) bits: the division-free
+// correctly rounded quotient, then rint by the rounding constant.
+__device__ __forceinline__ uint32_t code_bits(float x, float m, float s, float r) {
+  const float d = __fsub_rn(x, m);
+  const float q0 = __fmul_rn(d, r);
+  const float e = __fmaf_rn(-q0, s, d);
+  const float q1 = __fmaf_rn(e, r, q0);
+  return __float_as_uint(__fadd_rn(q1, kMagic));
+}
+
 // Second pass over one block: codes packed CPW per word, stored (words
 // shared with a neighbouring block updated atomically).  `row(t)` returns
-// channels c8..c8+7 of token t and `elem(t, i)` channel c8 + i.  The fast
-// path is branch-free so that the 8 x CPW codes of a word are independent;
-// codes near a rounding tie are marked in a bit mask and recomputed after.
+// channels c8..c8+7 of token t and `elem(t, i)` channel c8 + i.  Branch-free
+// per code, so the 8 x CPW codes of a word are independent.
 template <int BITS, int G, class RowFn, class ElemFn>
 __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, const float* cell_s, const float* cell_r,
-                                           const float* cell_nmr, const float* cell_m, const float* cell_dl, RowFn row,
-                                           ElemFn elem) {
+                                           const float* cell_m, const uint32_t* cell_fast, RowFn row, ElemFn elem) {
   constexpr int CPW = 32 / BITS;
   constexpr int TPR = G / 8;
   constexpr int RPI = kThreads / TPR;
@@ -198,12 +204,14 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
   const int tid = threadIdx.x;
   const int c8 = (tid % TPR) * 8;
   const int sub = tid / TPR;
-  float cr[8], cn[8], cd[8];
+  float cm[8], cs[8], cr[8];
+  uint32_t slow = 0;  // channels whose codes take the division
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    cm[i] = cell_m[c8 + i];
+    cs[i] = cell_s[c8 + i];
     cr[i] = cell_r[c8 + i];
-    cn[i] = cell_nmr[c8 + i];
-    cd[i] = cell_dl[c8 + i];
+    slow |= (cell_fast[c8 + i] ? 0u : 1u) << i;
   }
   const int w_lo = it.t0 / CPW;
   const int w_hi = (it.t1 - 1) / CPW;
@@ -212,15 +220,15 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
   for (int w = w_lo + sub; w <= w_hi; w += RPI) {
     const int tw = w * CPW;
     const bool full = (tw >= it.t0) && (tw + CPW <= it.t1);  // every slot in this block
-    uint32_t word[8], exc[8];
+    uint32_t word[8];
     uint32_t own = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word[i] = exc[i] = 0;
+    for (int i = 0; i < 8; ++i) word[i] = 0;
     if (full) {
       // the common case: every row of the word first (loads in flight
-      // together), then the codes.  yq = 1.5 2^23 + q holds q in its low
-      // bits, so the word is sum_j bits(yq_j) 2^(j b) minus the constant
-      // sum_j bits(1.5 2^23) 2^(j b): one integer multiply-add per code.
+      // together), then the codes.  The code bits are 1.5 2^23 + q, so the
+      // word is sum_j bits_j 2^(j b) minus the constant sum_j bits(1.5 2^23)
+      // 2^(j b): one integer multiply-add per code.
       own = 0xFFFFFFFFu;
       constexpr int CH = CPW > 4 ? 4 : CPW;  // rows loaded together
 #pragma unroll
@@ -236,14 +244,7 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
           float f[8];
           bf16x8_to_f32(v[u], f);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float y = __fmaf_rn(f[i], cr[i], cn[i]);
-            const float yq = __fadd_rn(y, kMagic);
-            const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
-            // false near a tie or when y is not finite; the field is rewritten below
-            exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
-            word[i] += __float_as_uint(yq) << (j * BITS);
-          }
+          for (int i = 0; i < 8; ++i) word[i] += code_bits(f[i], cm[i], cs[i], cr[i]) << (j * BITS);
         }
       }
       constexpr uint32_t kMagicSum = [] {
@@ -263,26 +264,22 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
         float f[8];
         bf16x8_to_f32(row(t), f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float y = __fmaf_rn(f[i], cr[i], cn[i]);
-          const float yq = __fadd_rn(y, kMagic);
-          const float e = __fsub_rn(y, __fsub_rn(yq, kMagic));
-          exc[i] |= (fabsf(e) <= cd[i]) ? 0u : (1u << j);
-          word[i] |= (__float_as_uint(yq) & MASK) << (j * BITS);
-        }
+        for (int i = 0; i < 8; ++i) word[i] |= (code_bits(f[i], cm[i], cs[i], cr[i]) & MASK) << (j * BITS);
       }
     }
+    if (slow != 0u) {
+      // cells outside the division-free quotient's range: the definition
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      // codes near a rounding tie: the exact quotient decides.  (A cell with
-      // a non-finite y has every code of the word marked; the sum above may
-      // then have carried into the unused high bits, which are cleared.)
-      if (exc[i] != 0u) word[i] &= USED;
-      while (exc[i] != 0u) {
-        const int j = __ffs(exc[i]) - 1;
-        exc[i] &= exc[i] - 1u;
-        const uint32_t q = exact_code<BITS>(elem(tw + j, i), cell_m[c8 + i], cell_s[c8 + i]);
-        word[i] = (word[i] & ~(MASK << (j * BITS))) | (q << (j * BITS));
+      for (int i = 0; i < 8; ++i) {
+        if (!((slow >> i) & 1u)) continue;
+        uint32_t wd = 0;
+#pragma unroll 1
+        for (int j = 0; j < CPW; ++j) {
+          const int t = tw + j;
+          if (t < it.t0 || t >= it.t1) continue;
+          wd |= exact_code<BITS>(elem(t, i), cm[i], cs[i]) << (j * BITS);
+        }
+        word[i] = wd;
       }
     }
     if (tw >= it.t0 && tw < it.t1) own |= ~USED;  // unused high bits belong to slot 0's block
@@ -311,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_co
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ float red_mn[kWarps][G];
   __shared__ float red_mx[kWarps][G];
-  __shared__ float cell_s[G], cell_r[G], cell_nmr[G], cell_m[G], cell_dl[G];
+  __shared__ float cell_s[G], cell_r[G], cell_m[G];
+  __shared__ uint32_t cell_fast[G];
   const int tid = threadIdx.x;
   const int oct = tid % TPR;
   const int c8 = oct * 8;
@@ -340,19 +338,22 @@ __global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_co
     }
   }
   float m0 = 0.0f, m1 = 0.0f;
-  if (block_reduce<G>(p, red_mn, red_mx, m0, m1) && tid == 0) report(a.dev_status, VARQ_DEV_NONFINITE);
-  if (tid < G) cell_constants<BITS, G>(a, it, m0, m1, cell_s, cell_r, cell_nmr, cell_m, cell_dl);
+  block_reduce<G>(p, red_mn, red_mx, m0, m1);
+  if (tid < G) {
+    if (!(fabsf(m0) <= 3.4e38f && fabsf(m1) <= 3.4e38f)) report(a.dev_status, VARQ_DEV_NONFINITE);
+    cell_constants<BITS, G>(a, it, m0, m1, cell_s, cell_r, cell_m, cell_fast);
+  }
   __syncthreads();
 
   // ---- pass 2: codes ----
   if (STAGED) {
     const __nv_bfloat16* st16 = reinterpret_cast<const __nv_bfloat16*>(stage);
     pack_block<BITS, G>(
-        a, it, cell_s, cell_r, cell_nmr, cell_m, cell_dl, [&](int t) { return stage[(t - it.t0) * TPR + oct]; },
+        a, it, cell_s, cell_r, cell_m, cell_fast, [&](int t) { return stage[(t - it.t0) * TPR + oct]; },
         [&](int t, int i) { return __bfloat162float(st16[(t - it.t0) * G + c8 + i]); });
   } else {
     pack_block<BITS, G>(
-        a, it, cell_s, cell_r, cell_nmr, cell_m, cell_dl,
+        a, it, cell_s, cell_r, cell_m, cell_fast,
         [&](int t) { return __ldg(reinterpret_cast<const uint4*>(it.xg + int64_t(t - it.t0) * a.st + c8)); },
         [&](int t, int i) { return __bfloat162float(it.xg[int64_t(t - it.t0) * a.st + c8 + i]); });
   }
