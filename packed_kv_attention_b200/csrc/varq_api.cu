@@ -116,6 +116,7 @@ int varq_quantize_pack_launches(const varq_cache_layout* L, int first_block, int
   std::memset(&a, 0, sizeof(a));
   a.first_block = first_block;
   a.n_blocks = n_blocks;
+  a.bits = L->bits;
   std::memcpy(a.block_start, L->block_start, sizeof(a.block_start));
   return varq::quant_pack_launch_count(a);
 }

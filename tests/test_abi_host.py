@@ -230,10 +230,12 @@ def test_status_strings():
 
 
 def test_quantize_pack_launch_count():
-    """One launch per group of blocks of similar length (<= 256 tokens, longer)."""
-    L = V.varq_cache_alloc(1, 1, 128, 4, [0, 1, 5, 21, 300, 1000])
+    """One launch per class of block length: <= 256 tokens (staged in shared
+    memory), longer (two passes through L2)."""
+    L = V.varq_cache_alloc(1, 1, 128, 4, [0, 1, 5, 21, 300, 1000, 9192])
     assert V.varq_quantize_pack_launches(L) == 2
     assert V.varq_quantize_pack_launches(L, 0, 3) == 1
     assert V.varq_quantize_pack_launches(L, 3, 2) == 1
+    assert V.varq_quantize_pack_launches(L, 2, 3) == 2
     with pytest.raises(V.VarqError):
-        V.varq_quantize_pack_launches(L, 4, 2)
+        V.varq_quantize_pack_launches(L, 4, 3)

@@ -41,6 +41,9 @@ SCHEDULES = {
     "one_block": [77],
     "unit_blocks": [1] * 12,
     "frames": [160, 160, 160],
+    # long blocks (two passes through L2) with ragged word boundaries
+    "long_ragged": [3, 300, 1001, 2049, 77, 4100],
+    "long_9k": [9001, 5],
 }
 
 
