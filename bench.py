@@ -730,6 +730,64 @@ def config_of(w, args):
             "l2": "inputs larger than L2 (bf16 K+V of the step exceed 126 MB)"}
 
 
+def profile_case(name):
+    """One small case of one kernel, for an ncu capture (`-k` the kernel,
+    `-s` the warm-up launches): inputs above the 126 MB L2 but a few hundred
+    MB on the device, three launches of the kernel, then exit."""
+    from packed_kv_attention_b200 import varq as V
+    dev = torch.device("cuda:0")
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    if name == "attn_sk_sweep_int4_lq16":
+        # swap-AB split-KV kernel: a quarter of the sweep cache (B2 H32 T16384 D128), INT4, Lq 16
+        w = synth.WORKLOADS["sweep"]
+        data = synth.make_inputs(w, lq=16, seed=3, device=dev, batch=2)
+        L = V.varq_cache_alloc(2, w.heads, w.head_dim, 4, data["block_start"])
+        kp, km = V.alloc_cache(L, dev)
+        vp, vm = V.alloc_cache(L, dev)
+        V.varq_quantize_pack(L, data["k"], kp, km)
+        V.varq_quantize_pack(L, data["v"], vp, vm)
+        q = data["q"].contiguous()
+        o = torch.empty_like(q)
+        ws = torch.empty(max(V.varq_packed_attention_workspace(L, 16, w.n_blocks) // 4, 1), dtype=torch.float32,
+                         device=dev)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            V.varq_packed_attention(L, q, kp, km, vp, vm, o, workspace=ws, dev_status=st)
+    elif name == "quant_pack_sweep_b1_int4":
+        # quantize+pack of one tensor [1, 32, 16384, 128] (128 MiB) in 16 blocks of 1,024 tokens, INT4
+        sizes = (1024,) * 16
+        g = torch.Generator(device=dev)
+        g.manual_seed(0)
+        x = synth.kv_cache(g, 1, 32, sizes, 128, 8, 10.0, 80.0, device=dev)
+        L = V.varq_cache_alloc(1, 32, 128, 4, synth.block_starts(sizes))
+        kp, km = V.alloc_cache(L, dev)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            V.varq_quantize_pack(L, x, kp, km, dev_status=st)
+    elif name == "attn_tc2_self_forcing_b2_schedule":
+        # paired-CTA kernel, pre-RoPE keys rotated from the 3D schedule: two of the twelve
+        # sequences of the Self-Forcing-like layer (B2 H12 T32760 D128, Lq 4680), INT4
+        w = synth.WORKLOADS["self_forcing"]
+        data = synth.make_inputs(w, lq=w.lq[-1], seed=4, device=dev, batch=2)
+        L = V.varq_cache_alloc(2, w.heads, w.head_dim, 4, data["block_start"])
+        kp, km = V.alloc_cache(L, dev)
+        vp, vm = V.alloc_cache(L, dev)
+        V.varq_quantize_pack(L, data["k"], kp, km)
+        V.varq_quantize_pack(L, data["v"], vp, vm)
+        o = torch.empty_like(data["q"])
+        rope = V.Rope3d.make(1560, 52, synth.rope_axis_pairs(w.head_dim))
+        torch.cuda.synchronize()
+        for _ in range(3):
+            V.varq_packed_attention_rope3d(L, data["q"], kp, km, vp, vm, o, rope, dev_status=st)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "device_status": int(st.item())}))
+
+
+PROFILE_CASES = ("attn_sk_sweep_int4_lq16", "quant_pack_sweep_b1_int4", "attn_tc2_self_forcing_b2_schedule")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -745,7 +803,12 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements (unpack, split-KV, pre-RoPE)")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES,
+                    help="run one small case of one kernel for an ncu capture, then exit (no JSON line)")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     w = synth.WORKLOADS[args.workload]
     if args.lq <= 0:
         args.lq = w.lq[-1]
