@@ -13,12 +13,13 @@
 //     block is staged in shared memory while its min/max is reduced, and the
 //     codes are computed from shared memory.
 //   - Longer blocks: G = 16 (32-byte row pieces, one DRAM sector).  The first
-//     pass streams the rows from HBM (eight 16-byte loads in flight per thread)
-//     reducing min/max; the second pass re-reads the same rows, which the few
-//     hundred resident CTAs' footprints (<= ~150 KB each) keep in the 126 MB L2.
-// Min/max are reduced on packed bf16x2 with NaN-propagating instructions,
-// then with warp shuffles over the lanes that hold the same channels, then a
-// shared-memory tree across warps.
+//     pass streams the rows from HBM (four 16-byte loads in flight per thread,
+//     six CTAs per SM) reducing min/max; the second pass re-reads the same
+//     rows, which the resident CTAs' footprints (<= ~150 KB each) keep in the
+//     126 MB L2, four channels per thread.
+// Min/max are taken on packed bf16x2 with NaN-propagating instructions and
+// reduced as packed pairs by warp shuffles over the lanes that hold the same
+// channels, then across warps in shared memory.
 //
 // Arithmetic is the exact fp32 definition:
 //   s = fp32(fp32(max - min) / (2^b - 1)),  q = rint(fp32(fp32(x - min) / s)).
@@ -33,6 +34,7 @@
 // below 2^-100 (so that e could fall below the subnormal grid) -- take
 // __fdiv_rn for every code.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -45,6 +47,12 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 8;          // rows per thread loaded back to back
 constexpr int kStageRows = 256;    // blocks up to this length are staged in shared memory
+// The long-block kernel: six resident CTAs per SM (40 registers; the code pass
+// takes four channels a thread) and four 16-byte loads in flight per thread in
+// the min/max pass -- measured best of 4-6 CTAs x 4-8 loads on the 1 GiB sweep
+// and the Infinity-8B-like cache.
+constexpr int kLongMinBlocks = 6;
+constexpr int kLongBatch = 4;
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer (ties to even)
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
@@ -190,61 +198,78 @@ __device__ __forceinline__ uint32_t code_bits(float x, float m, float s, float r
 }
 
 // Second pass over one block: codes packed CPW per word, stored (words
-// shared with a neighbouring block updated atomically).  `row(t)` returns
-// channels c8..c8+7 of token t and `elem(t, i)` channel c8 + i.  Branch-free
-// per code, so the 8 x CPW codes of a word are independent.
-template <int BITS, int G, class RowFn, class ElemFn>
+// shared with a neighbouring block updated atomically).  Each thread codes
+// VEC channels (c0 .. c0 + VEC - 1) of one word at a time; `row(t, c0)`
+// returns those channels of token t (uint4 for 8, uint2 for 4) and
+// `elem(t, c)` channel c.  Branch-free per code, so the VEC x CPW codes of a
+// word are independent.
+template <int VEC>
+using RowT = typename std::conditional<VEC == 8, uint4, uint2>::type;
+
+template <int VEC>
+__device__ __forceinline__ void row_to_f32(const RowT<VEC>& v, float (&f)[VEC]) {
+  if constexpr (VEC == 8) {
+    bf16x8_to_f32(v, f);
+  } else {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  }
+}
+
+template <int BITS, int G, int VEC, class RowFn, class ElemFn>
 __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, const float* cell_s, const float* cell_r,
                                            const float* cell_m, const uint32_t* cell_fast, RowFn row, ElemFn elem) {
   constexpr int CPW = 32 / BITS;
-  constexpr int TPR = G / 8;
+  constexpr int TPR = G / VEC;
   constexpr int RPI = kThreads / TPR;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   constexpr uint32_t USED = uint32_t(CPW * BITS) == 32u ? 0xFFFFFFFFu : ((1u << (CPW * BITS)) - 1u);
   const int tid = threadIdx.x;
-  const int c8 = (tid % TPR) * 8;
+  const int c0 = (tid % TPR) * VEC;
   const int sub = tid / TPR;
-  float cm[8], cs[8], cr[8];
+  float cm[VEC], cs[VEC], cr[VEC];
   uint32_t slow = 0;  // channels whose codes take the division
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    cm[i] = cell_m[c8 + i];
-    cs[i] = cell_s[c8 + i];
-    cr[i] = cell_r[c8 + i];
-    slow |= (cell_fast[c8 + i] ? 0u : 1u) << i;
+  for (int i = 0; i < VEC; ++i) {
+    cm[i] = cell_m[c0 + i];
+    cs[i] = cell_s[c0 + i];
+    cr[i] = cell_r[c0 + i];
+    slow |= (cell_fast[c0 + i] ? 0u : 1u) << i;
   }
   const int w_lo = it.t0 / CPW;
   const int w_hi = (it.t1 - 1) / CPW;
   const bool last_block = (it.t1 == a.n_tokens);
-  uint32_t* pk = a.packed + (int64_t(it.b) * a.heads + it.h) * a.words_per_row * a.head_dim + it.g * G + c8;
+  uint32_t* pk = a.packed + (int64_t(it.b) * a.heads + it.h) * a.words_per_row * a.head_dim + it.g * G + c0;
   for (int w = w_lo + sub; w <= w_hi; w += RPI) {
     const int tw = w * CPW;
     const bool full = (tw >= it.t0) && (tw + CPW <= it.t1);  // every slot in this block
-    uint32_t word[8];
+    uint32_t word[VEC];
     uint32_t own = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word[i] = 0;
+    for (int i = 0; i < VEC; ++i) word[i] = 0;
     if (full) {
-      // the common case: every row of the word first (loads in flight
-      // together), then the codes.  The code bits are 1.5 2^23 + q, so the
-      // word is sum_j bits_j 2^(j b) minus the constant sum_j bits(1.5 2^23)
-      // 2^(j b): one integer multiply-add per code.
+      // the common case: rows of the word loaded together, then the codes.
+      // The code bits are 1.5 2^23 + q, so the word is sum_j bits_j 2^(j b)
+      // minus the constant sum_j bits(1.5 2^23) 2^(j b): one integer
+      // multiply-add per code.
       own = 0xFFFFFFFFu;
       constexpr int CH = CPW > 4 ? 4 : CPW;  // rows loaded together
 #pragma unroll
       for (int j0 = 0; j0 < CPW; j0 += CH) {
-        uint4 v[CH];
+        RowT<VEC> v[CH];
 #pragma unroll
         for (int u = 0; u < CH; ++u)
-          if (j0 + u < CPW) v[u] = row(tw + j0 + u);
+          if (j0 + u < CPW) v[u] = row(tw + j0 + u, c0);
 #pragma unroll
         for (int u = 0; u < CH; ++u) {
           const int j = j0 + u;
           if (j >= CPW) break;
-          float f[8];
-          bf16x8_to_f32(v[u], f);
+          float f[VEC];
+          row_to_f32<VEC>(v[u], f);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) word[i] += code_bits(f[i], cm[i], cs[i], cr[i]) << (j * BITS);
+          for (int i = 0; i < VEC; ++i) word[i] += code_bits(f[i], cm[i], cs[i], cr[i]) << (j * BITS);
         }
       }
       constexpr uint32_t kMagicSum = [] {
@@ -253,7 +278,7 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
         return k;
       }();
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word[i] -= kMagicSum;
+      for (int i = 0; i < VEC; ++i) word[i] -= kMagicSum;
     } else {
 #pragma unroll
       for (int j = 0; j < CPW; ++j) {
@@ -261,23 +286,23 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
         const bool mine = t >= it.t0 && t < it.t1;
         if (mine || (last_block && t >= it.t1)) own |= MASK << (j * BITS);
         if (!mine) continue;
-        float f[8];
-        bf16x8_to_f32(row(t), f);
+        float f[VEC];
+        row_to_f32<VEC>(row(t, c0), f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word[i] |= (code_bits(f[i], cm[i], cs[i], cr[i]) & MASK) << (j * BITS);
+        for (int i = 0; i < VEC; ++i) word[i] |= (code_bits(f[i], cm[i], cs[i], cr[i]) & MASK) << (j * BITS);
       }
     }
     if (slow != 0u) {
       // cells outside the division-free quotient's range: the definition
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < VEC; ++i) {
         if (!((slow >> i) & 1u)) continue;
         uint32_t wd = 0;
 #pragma unroll 1
         for (int j = 0; j < CPW; ++j) {
           const int t = tw + j;
           if (t < it.t0 || t >= it.t1) continue;
-          wd |= exact_code<BITS>(elem(t, i), cm[i], cs[i]) << (j * BITS);
+          wd |= exact_code<BITS>(elem(t, c0 + i), cm[i], cs[i]) << (j * BITS);
         }
         word[i] = wd;
       }
@@ -286,10 +311,10 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
     uint32_t* dst = pk + int64_t(w) * a.head_dim;
     if (own == 0xFFFFFFFFu) {
       reinterpret_cast<uint4*>(dst)[0] = make_uint4(word[0], word[1], word[2], word[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(word[4], word[5], word[6], word[7]);
+      if constexpr (VEC == 8) reinterpret_cast<uint4*>(dst)[1] = make_uint4(word[4], word[5], word[6], word[7]);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < VEC; ++i) {
         atomicAnd(dst + i, ~own);
         atomicOr(dst + i, word[i] & own);
       }
@@ -302,7 +327,7 @@ __device__ __forceinline__ void pack_block(const QuantArgs& a, const Item& it, c
 // One CTA per (b, h, block, G channels).  STAGED: the block sits in shared
 // memory between the passes; otherwise the second pass re-reads it (L2).
 template <int BITS, int G, bool STAGED>
-__global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, STAGED ? 4 : kLongMinBlocks) quant_pack_kernel(const __grid_constant__ QuantArgs a) {
   constexpr int TPR = G / 8;
   constexpr int RPI = kThreads / TPR;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -321,15 +346,16 @@ __global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_co
   // ---- pass 1: min / max, kBatch 16-byte loads in flight per thread ----
   Partial p;
   p.init();
-  for (int base = 0; base < rows; base += RPI * kBatch) {
-    uint4 v[kBatch];
+  constexpr int NB = STAGED ? kBatch : kLongBatch;  // 16-byte loads in flight per thread
+  for (int base = 0; base < rows; base += RPI * NB) {
+    uint4 v[NB];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+    for (int u = 0; u < NB; ++u) {
       const int r = base + sub + u * RPI;
       if (r < rows) v[u] = __ldg(reinterpret_cast<const uint4*>(it.xg + int64_t(r) * a.st + c8));
     }
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+    for (int u = 0; u < NB; ++u) {
       const int r = base + sub + u * RPI;
       if (r < rows) {
         if (STAGED) stage[r * TPR + oct] = v[u];
@@ -346,16 +372,19 @@ __global__ void __launch_bounds__(kThreads, 4) quant_pack_kernel(const __grid_co
   __syncthreads();
 
   // ---- pass 2: codes ----
-  if (STAGED) {
+  if constexpr (STAGED) {
     const __nv_bfloat16* st16 = reinterpret_cast<const __nv_bfloat16*>(stage);
-    pack_block<BITS, G>(
-        a, it, cell_s, cell_r, cell_m, cell_fast, [&](int t) { return stage[(t - it.t0) * TPR + oct]; },
-        [&](int t, int i) { return __bfloat162float(st16[(t - it.t0) * G + c8 + i]); });
-  } else {
-    pack_block<BITS, G>(
+    pack_block<BITS, G, 8>(
         a, it, cell_s, cell_r, cell_m, cell_fast,
-        [&](int t) { return __ldg(reinterpret_cast<const uint4*>(it.xg + int64_t(t - it.t0) * a.st + c8)); },
-        [&](int t, int i) { return __bfloat162float(it.xg[int64_t(t - it.t0) * a.st + c8 + i]); });
+        [&](int t, int c) { return stage[(t - it.t0) * TPR + c / 8]; },
+        [&](int t, int c) { return __bfloat162float(st16[(t - it.t0) * G + c]); });
+  } else {
+    // four channels a thread: fewer registers, more resident warps to hide
+    // the re-reads' latency
+    pack_block<BITS, G, 4>(
+        a, it, cell_s, cell_r, cell_m, cell_fast,
+        [&](int t, int c) { return __ldg(reinterpret_cast<const uint2*>(it.xg + int64_t(t - it.t0) * a.st + c)); },
+        [&](int t, int c) { return __bfloat162float(it.xg[int64_t(t - it.t0) * a.st + c]); });
   }
 }
 
