@@ -428,8 +428,8 @@ template <int BITS, bool ROPE, bool SCHED = false>
 cudaError_t launch_sk(const AttnArgs& a, cudaStream_t stream) {
   using C = SkCfg<BITS, 128>;
   auto kern = attn_sk_kernel<BITS, ROPE, SCHED>;
+  if (SCHED && !rope_table_fits(a, C::SMEM, kSmemMaxDynamic)) return cudaErrorInvalidConfiguration;
   const uint32_t smem = C::SMEM + (SCHED ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
-  if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const dim3 grid(unsigned(a.n_splits), unsigned(a.heads), unsigned(a.batch));

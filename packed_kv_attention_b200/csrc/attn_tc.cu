@@ -299,8 +299,8 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   // every CTA allocates all 512 TMEM columns: ask for enough shared memory
   // that no second CTA is placed on the SM to wait for them (plus the rotary
   // table of rope mode 2, which must fit)
+  if (SCHED && !rope_table_fits(a, C::SMEM, kSmemMaxDynamic)) return cudaErrorInvalidConfiguration;
   const uint32_t extra = SCHED ? rope_table_bytes(a) : 0u;
-  if (C::SMEM + extra > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   const uint32_t smem = std::max<uint32_t>(C::SMEM + extra, kSmemUsable / 2 + 1024);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;

@@ -640,8 +640,8 @@ template <int BITS, int D, int NQ, bool ROPE, bool SCHED = false>
 cudaError_t launch_tc2(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg2<BITS, D, NQ>;
   auto kern = attn_tc2_kernel<BITS, D, NQ, ROPE, SCHED>;
+  if (SCHED && !rope_table_fits(a, C::SMEM, kSmemMaxDynamic)) return cudaErrorInvalidConfiguration;
   const uint32_t smem = C::SMEM + (SCHED ? rope_table_bytes(a) : 0u);  // + the rotary table of rope mode 2
-  if (smem > kSmemMaxDynamic) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int pairs = (a.lq + 2 * NQ * BM - 1) / (2 * NQ * BM) * (a.kv_split ? a.n_splits : 1);

@@ -175,11 +175,19 @@ inline void set_rope_lens(AttnArgs& a) {
 }
 // Bytes of the per-CTA rotary table of rope_mode 2 (0 otherwise): float2
 // (cos, sin) entries, per pair, along its axis.
+// Saturates at UINT32_MAX (a schedule whose table could never fit).
 inline uint32_t rope_table_bytes(const AttnArgs& a) {
   if (a.rope_mode != 2) return 0;
   const int64_t n = int64_t(a.rope_len[0]) * a.rope_pairs[0] + int64_t(a.rope_len[1]) * a.rope_pairs[1] +
                     int64_t(a.rope_len[2]) * a.rope_pairs[2];
-  return uint32_t(((n * 8) + 127) / 128 * 128);
+  const int64_t bytes = (n * 8 + 127) / 128 * 128;
+  return bytes > int64_t(UINT32_MAX) ? UINT32_MAX : uint32_t(bytes);
+}
+// Whether `base` bytes of a kernel's own shared memory plus the rotary table
+// fit in one CTA's dynamic shared memory (`limit`), without wrapping.
+inline bool rope_table_fits(const AttnArgs& a, uint32_t base, uint32_t limit) {
+  const uint32_t t = rope_table_bytes(a);
+  return base <= limit && t <= limit - base;
 }
 
 // Tensor-core attention; with kv_split, the split-KV form plus its combine.

@@ -184,6 +184,10 @@ def test_rope3d_attention_errors():
     # holds next to the kernel's buffers: refused before any launch
     long_cache = V.varq_cache_alloc(1, 1, 128, 4, [0, 50000, 100000])
     assert call(frame=1, gw=1, path=1, nc=2, lay=long_cache) == UNSUPPORTED
+    # a table beyond 4 GB must not wrap into a size that seems to fit
+    huge_cache = V.varq_cache_alloc(1, 1, 128, 4, [0, 30_000_000])
+    assert call(frame=1, gw=1, path=1, nc=1, lay=huge_cache) == UNSUPPORTED
+    assert call(frame=1, gw=1, path=2, lq=4, nc=1, lay=huge_cache) in (UNSUPPORTED, WORKSPACE)
 
 
 def test_dense_attention_errors():
