@@ -809,13 +809,43 @@ def profile_case(name):
         torch.cuda.synchronize()
         for _ in range(3):
             V.varq_packed_attention_rope3d(L, data["q"], kp, km, vp, vm, o, rope, dev_status=st)
+    elif name == "unpack_dequant_sweep_b1_int4":
+        # standalone unpack+dequant of one packed tensor [1, 32, 16384, 128] to bf16, INT4
+        sizes = (1024,) * 16
+        g = torch.Generator(device=dev)
+        g.manual_seed(0)
+        x = synth.kv_cache(g, 1, 32, sizes, 128, 8, 10.0, 80.0, device=dev)
+        L = V.varq_cache_alloc(1, 32, 128, 4, synth.block_starts(sizes))
+        kp, km = V.alloc_cache(L, dev)
+        V.varq_quantize_pack(L, x, kp, km, dev_status=st)
+        out = torch.empty_like(x)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            V.varq_unpack_dequant(L, kp, km, out)
+    elif name == "attn_decode_sweep_int4_lq1":
+        # CUDA-core split-KV decode: a quarter of the sweep cache (B2 H32 T16384 D128), INT4, Lq 1
+        w = synth.WORKLOADS["sweep"]
+        data = synth.make_inputs(w, lq=1, seed=3, device=dev, batch=2)
+        L = V.varq_cache_alloc(2, w.heads, w.head_dim, 4, data["block_start"])
+        kp, km = V.alloc_cache(L, dev)
+        vp, vm = V.alloc_cache(L, dev)
+        V.varq_quantize_pack(L, data["k"], kp, km)
+        V.varq_quantize_pack(L, data["v"], vp, vm)
+        q = data["q"].contiguous()
+        o = torch.empty_like(q)
+        ws = torch.empty(max(V.varq_packed_attention_workspace(L, 1, w.n_blocks) // 4, 1), dtype=torch.float32,
+                         device=dev)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            V.varq_packed_attention(L, q, kp, km, vp, vm, o, workspace=ws, dev_status=st)
     else:
         raise SystemExit(f"unknown profile case {name}")
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": name, "device_status": int(st.item())}))
 
 
-PROFILE_CASES = ("attn_sk_sweep_int4_lq16", "quant_pack_sweep_b1_int4", "attn_tc2_self_forcing_b2_schedule")
+PROFILE_CASES = ("attn_sk_sweep_int4_lq16", "quant_pack_sweep_b1_int4", "attn_tc2_self_forcing_b2_schedule",
+                 "unpack_dequant_sweep_b1_int4", "attn_decode_sweep_int4_lq1")
 
 
 def main(argv=None):
