@@ -969,6 +969,7 @@ def main(argv=None):
         pipe = Pipeline(w, args.bits, args.lq, dev)
     if not args.no_e2e:
         e2e_ms, h2d, d2h, same = time_e2e(pipe, max(4, args.steps), 2, stream)
+        e2e_ms = max_over_ranks(e2e_ms, dev, dist_ok)  # every rank runs this section
         line["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                        "copies": "own streams, overlapping the neighbouring steps' kernels (two buffer sets)",
