@@ -249,7 +249,8 @@ typedef struct varq_rope3d {
  * mode with the rotation angles computed from token positions instead of read
  * from [T, D/2] tables ([PAGE] "The block axis", Eq. 3: RoPE rotates each
  * (2i, 2i+1) key pair; Appendix F: keys quantized before RoPE).  Every other
- * argument as varq_packed_attention (whose rope_cos / rope_sin this replaces).
+ * argument as varq_packed_attention (whose rope_cos / rope_sin this replaces);
+ * `rope` is a host pointer, read before the call returns (the caller keeps it).
  * Each CTA tabulates cos and sin of the angles its tokens use (the frames of
  * its part of the cache, every row, every column) in shared memory,
  * computed in double precision and rounded to fp32 -- the values a host
