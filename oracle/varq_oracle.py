@@ -46,6 +46,13 @@ R7  Pre-RoPE key mode: the dequantized key pair (2i, 2i+1) is rotated by the
     caller's per-token angle table ([PAGE] "The block axis", Eq. 3: RoPE
     rotates each (2i, 2i+1) pair; Appendix F: pre-RoPE quantization is an
     option, post-RoPE the default).
+R8  3D rotary schedule of the video models: token t lies in latent frame
+    t // F, at row (t mod F) // W and column t mod W (F tokens per frame, W
+    per row); key pair i belongs to the frame, row or column axis by the
+    split (P0, P1, P2) and, as pair j of its axis's n, turns by
+    position * base^(-j/n).  The angles are taken in fp64 and cos, sin rounded
+    to fp32, as a table would be stored.  The pages give the 1,560-token frame
+    ([README] "Configs"); the per-axis split and the base are this build's.
 """
 from __future__ import annotations
 
@@ -58,7 +65,7 @@ __all__ = [
     "codes_per_word", "words_per_row", "bf16_to_f32", "f32_to_bf16",
     "f32_to_f16_bits", "f16_bits_to_f32", "quantize_cell", "quantize",
     "meta_words", "pack", "unpack", "token_block", "dequantize",
-    "rope_rotate", "attention", "cache_layout", "kv_reduction",
+    "rope_rotate", "rope_schedule_tables", "attention", "cache_layout", "kv_reduction",
 ]
 
 
@@ -230,6 +237,24 @@ def rope_rotate(k: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
     out[..., 0::2] = a * c - b * s
     out[..., 1::2] = a * s + b * c
     return out
+
+
+def rope_schedule_tables(n_tokens: int, frame_tokens: int, grid_w: int, pairs: Sequence[int],
+                         base: float = 10000.0):
+    """R8: fp32 ``cos, sin [T, sum(pairs)]`` of the 3D (frame, row, column)
+    rotary schedule ([PAGE] "The block axis", Eq. 3: RoPE rotates each
+    (2i, 2i+1) key pair by its angle)."""
+    t = np.arange(n_tokens, dtype=np.int64)
+    frame = t // frame_tokens
+    in_frame = t % frame_tokens
+    row = in_frame // grid_w
+    col = in_frame % grid_w
+    cols = []
+    for position, n in ((frame, pairs[0]), (row, pairs[1]), (col, pairs[2])):
+        for j in range(n):
+            cols.append(position.astype(np.float64) * float(base) ** (-j / n))
+    ang = np.stack(cols, axis=1) if cols else np.zeros((n_tokens, 0))
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
 
 
 def attention(q_bf16: np.ndarray, k_hat_bf16: np.ndarray, v_hat_bf16: np.ndarray,

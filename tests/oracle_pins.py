@@ -477,6 +477,42 @@ def check_attention_rope_mode(O, seed=12):
     assert np.allclose(c, ref, atol=1e-12)
 
 
+def check_rope_schedule(O):
+    """R8 against positions worked out by hand and the schedule's structure."""
+    # F = 6 tokens per frame on a 3-wide grid (2 rows), pairs (2, 1, 1), base 10000.
+    # Token 7: frame 1, in-frame position 1 -> row 0, column 1.  Its angles:
+    # frame pairs 1 * 10000^0 = 1 and 1 * 10000^(-1/2) = 0.01; row pair 0 * 1 = 0;
+    # column pair 1 * 1 = 1.  Token 11: frame 1, position 5 -> row 1, column 2:
+    # angles 1, 0.01, 1, 2.  Token 26: frame 4 (frames count over the whole cache,
+    # not per chunk), position 2 -> row 0, column 2: angles 4, 0.04, 0, 2.
+    cos, sin = O.rope_schedule_tables(30, 6, 3, (2, 1, 1), 10000.0)
+    for t, angles in ((7, (1.0, 0.01, 0.0, 1.0)), (11, (1.0, 0.01, 1.0, 2.0)), (0, (0.0, 0.0, 0.0, 0.0)),
+                      (3, (0.0, 0.0, 1.0, 0.0)), (26, (4.0, 0.04, 0.0, 2.0))):
+        want_c = np.array([math.cos(x) for x in angles], np.float32)
+        want_s = np.array([math.sin(x) for x in angles], np.float32)
+        assert np.array_equal(cos[t], want_c) and np.array_equal(sin[t], want_s), t
+    # structure on the 1,560-token frames of the next-frame workloads (30 x 52, 22:21:21)
+    F, W, P = 1560, 52, (22, 21, 21)
+    T = 3 * F + 100
+    cos, sin = O.rope_schedule_tables(T, F, W, P)
+    fr, rw, cl = slice(0, 22), slice(22, 43), slice(43, 64)
+    t = np.arange(T)
+    # frame pairs change only at frame boundaries, row pairs only at row boundaries
+    same_frame = (t[1:] // F) == (t[:-1] // F)
+    assert np.array_equal(cos[1:, fr][same_frame], cos[:-1, fr][same_frame])
+    same_row = (t[1:] // W) == (t[:-1] // W)
+    assert np.array_equal(cos[1:, rw][same_row], cos[:-1, rw][same_row])
+    # rows and columns repeat every frame, columns every row
+    assert np.array_equal(cos[F:2 * F, rw], cos[:F, rw]) and np.array_equal(sin[F:2 * F, cl], sin[:F, cl])
+    assert np.array_equal(cos[W:2 * W, cl], cos[:W, cl])
+    # frequencies: at position 1 the angle of pair j of an axis with n pairs is base^(-j/n)
+    for ax, n, tok in ((fr, 22, F), (rw, 21, W), (cl, 21, 1)):
+        ang = np.arctan2(sin[tok, ax].astype(np.float64), cos[tok, ax].astype(np.float64))
+        assert np.allclose(ang, 10000.0 ** (-np.arange(n) / n), rtol=1e-6, atol=1e-7), ax
+    # a rotation: cos^2 + sin^2 = 1 to fp32 rounding
+    assert np.allclose(cos.astype(np.float64) ** 2 + sin.astype(np.float64) ** 2, 1.0, atol=1e-6)
+
+
 ALL_CHECKS = [
     check_hand_quantize, check_bruteforce_codes, check_fp32_quotient_definition,
     check_cell_stats, check_bound,
@@ -485,5 +521,5 @@ ALL_CHECKS = [
     check_dequant_single_rounding, check_constant_block_dequant,
     check_kv_reduction_pages, check_layout_sizes,
     check_attention_closed_forms, check_attention_scipy, check_rope,
-    check_attention_rope_mode,
+    check_attention_rope_mode, check_rope_schedule,
 ]

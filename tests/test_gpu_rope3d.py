@@ -1,16 +1,18 @@
 """Pre-RoPE keys rotated in the kernel from the 3D (frame, row, column)
 schedule instead of host tables, against the fp64 CPU oracle.
 
-The oracle takes fp32 cos/sin tables built on the host from the same
-schedule (chunked frames of ``frame`` tokens on a ``grid_w``-wide grid, the
-pairs split between the axes as in the next-frame workloads); the kernel
-computes the angles itself from token indices.  Tolerances are those of the
-table form (the LSE bound covers the fp16 rounding of the rotated key).
+The oracle's own restatement of the schedule (``rope_schedule_tables``:
+frames of ``frame`` tokens on a ``grid_w``-wide grid, the pairs split between
+the axes as in the next-frame workloads) gives the fp32 cos/sin it rotates
+by; the kernel computes the angles itself from token indices.  Tolerances
+are those of the table form (the LSE bound covers the fp16 rounding of the
+rotated key).
 """
 import numpy as np
 import pytest
 import torch
 
+from oracle import varq_oracle as O
 from packed_kv_attention_b200 import synth
 from packed_kv_attention_b200 import varq as V
 
@@ -37,6 +39,11 @@ def _run_rope3d(L, k, v, q, n_cached, frame, grid_w, path=V.PATH_AUTO, scale=0.0
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     return out, lse
+
+
+def _schedule(n_tokens, D, frame, grid_w):
+    cos, sin = O.rope_schedule_tables(n_tokens, frame, grid_w, synth.rope_axis_pairs(D))
+    return torch.from_numpy(cos), torch.from_numpy(sin)
 
 
 def _inputs(B, H, D, sizes, lq, seed):
@@ -72,7 +79,7 @@ def test_rope3d_small(case):
     B, H = 2, 2
     bs = synth.block_starts(sizes)
     k, v, q = _inputs(B, H, D, sizes, lq, seed=D + bits + lq + frame)
-    cos, sin = synth.rope_tables_3d(sum(sizes), D, chunk=3 * frame, frame=frame, grid_w=grid_w)
+    cos, sin = _schedule(sum(sizes), D, frame, grid_w)
     L = V.varq_cache_alloc(B, H, D, bits, bs)
     out, lse = _run_rope3d(L, k, v, q, len(sizes), frame, grid_w, path=path)
     rows = np.arange(lq)
@@ -89,7 +96,7 @@ def test_rope3d_prefix_of_cache(path, lq):
     D, bits, sizes, frame, grid_w = 128, 4, [120, 120, 120, 120], 40, 8
     bs = synth.block_starts(sizes)
     k, v, q = _inputs(1, 2, D, sizes, lq, seed=11)
-    cos, sin = synth.rope_tables_3d(sum(sizes), D, chunk=120, frame=frame, grid_w=grid_w)
+    cos, sin = _schedule(sum(sizes), D, frame, grid_w)
     L = V.varq_cache_alloc(1, 2, D, bits, bs)
     out, lse = _run_rope3d(L, k, v, q, 3, frame, grid_w, path=path)
     rows = np.arange(lq)
@@ -105,7 +112,7 @@ def test_rope3d_matches_tables():
     D, bits, sizes, lq, frame, grid_w = 128, 4, [1560, 1560, 1560], 64, 1560, 52
     bs = synth.block_starts(sizes)
     k, v, q = _inputs(2, 3, D, sizes, lq, seed=5)
-    cos, sin = synth.rope_tables_3d(sum(sizes), D)
+    cos, sin = _schedule(sum(sizes), D, frame, grid_w)
     L = V.varq_cache_alloc(2, 3, D, bits, bs)
     for path, n in ((V.PATH_TENSOR, lq), (V.PATH_SPLIT, 16)):
         q = q[:, :, :n].contiguous()
@@ -135,8 +142,8 @@ def test_rope3d_full_size(name, bits, lq):
     bs = data["block_start"]
     L = V.varq_cache_alloc(w.batch, w.heads, w.head_dim, bits, bs)
     out, lse = _run_rope3d(L, data["k"], data["v"], data["q"], w.n_blocks, 1560, 52)
-    cos, sin = data["rope_cos"].cpu(), data["rope_sin"].cpu()
     del data["rope_cos"], data["rope_sin"]
+    cos, sin = _schedule(w.n_tokens, w.head_dim, 1560, 52)
     k, v, q = data["k"].cpu(), data["v"].cpu(), data["q"].cpu()
     rng = np.random.default_rng(2)
     for (b, h) in [(0, 0), (w.batch - 1, w.heads - 1)]:

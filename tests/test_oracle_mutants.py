@@ -40,6 +40,10 @@ MUTANTS = {
     "rope_pairs_halves": ("a = k[..., 0::2]\n    b = k[..., 1::2]",
                           "a = k[..., :k.shape[-1] // 2]\n    b = k[..., k.shape[-1] // 2:]"),
     "meta_two_bytes": ("meta = nb * 32.0", "meta = nb * 16.0"),
+    "schedule_row_column_swapped": ("    row = in_frame // grid_w\n    col = in_frame % grid_w",
+                                    "    row = in_frame % grid_w\n    col = in_frame // grid_w"),
+    "schedule_frequency_exponent": ("float(base) ** (-j / n)", "float(base) ** (-2 * j / n)"),
+    "schedule_frame_local": ("frame = t // frame_tokens", "frame = (t // frame_tokens) % 3"),
     "reduction_per_block_padding": ("words = words_per_row(t, bits) if whole_words else t / cpw",
                                     "words = words_per_row(t, bits) + nb - 1"),
 }
