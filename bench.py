@@ -50,7 +50,7 @@ METRIC = "fused packed-KV attention TFLOP/s and quant+pack GB/s at INT4/INT2 (% 
 # kernel.  Reported as the roofline "traffic" only while the kernel's sources
 # hash to the value they had when the counters were taken; otherwise null.
 MEASURED_TRAFFIC = {"workload": "infinity_8b", "bits": 4, "lq": 4096, "rope": False,
-                    "bytes": 154.422784e6 + 40.189184e6, "sources_sha256_16": "ffd494df80cb039a"}
+                    "bytes": 154.583552e6 + 40.038144e6, "sources_sha256_16": "7cfc2c2543c454d0"}
 TRAFFIC_SOURCES = ("packed_kv_attention_b200/csrc/attn_tc.cu", "packed_kv_attention_b200/csrc/attn_tc_common.cuh",
                    "packed_kv_attention_b200/csrc/common.cuh")
 
