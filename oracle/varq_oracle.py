@@ -52,7 +52,9 @@ R8  3D rotary schedule of the video models: token t lies in latent frame
     split (P0, P1, P2) and, as pair j of its axis's n, turns by
     position * base^(-j/n).  The angles are taken in fp64 and cos, sin rounded
     to fp32, as a table would be stored.  The pages give the 1,560-token frame
-    ([README] "Configs"); the per-axis split and the base are this build's.
+    ([README] "Configs") but not the per-axis split or the base; the split
+    P - 2*floor(P/3) : floor(P/3) : floor(P/3) of the P pairs and base 10000
+    are the plainest choice.
 """
 from __future__ import annotations
 
