@@ -150,3 +150,29 @@ def test_rope3d_full_size(name, bits, lq):
         rows = _sample_rows(lq, rng, 16)
         ref, ref_lse = _oracle_attention(k, v, q, bs, bits, w.n_blocks, b, h, rows, cos=cos, sin=sin)
         _check(out, lse, ref, ref_lse, b, h, rows)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("path,lq", [(V.PATH_TENSOR, 200), (V.PATH_SPLIT, 8)])
+def test_rope3d_beyond_fp16_range(bits, path, lq):
+    """The schedule form with keys whose cells reach 9e4 (INT2) to 4e5 (INT4),
+    inside the metadata limits, and queries up to ~6e5: both beyond the fp16
+    range of S = Q K^T in this mode, scaled by powers of two into it; a custom
+    softmax scale keeps the scores moderate."""
+    import math
+    D, frame, grid_w = 128, 40, 8
+    sizes = [120, 120, 120, 45]
+    bs = synth.block_starts(sizes)
+    k, v, q = _inputs(1, 2, D, sizes, lq, seed=31 + bits)
+    k = (k.float().abs() * 2.0 ** (11 if bits == 4 else 9)).to(torch.bfloat16)  # powers of two: exact
+    q = (q.float() * 2.0 ** 17).to(torch.bfloat16)
+    scale = 2.0 ** -28 / math.sqrt(D) * (4.0 if bits == 2 else 1.0)
+    assert float(k.float().abs().max()) > 65504 and float(q.float().abs().max()) > 65504
+    cos, sin = _schedule(sum(sizes), D, frame, grid_w)
+    L = V.varq_cache_alloc(1, 2, D, bits, bs)
+    out, lse = _run_rope3d(L, k, v, q, len(sizes), frame, grid_w, path=path, scale=scale)
+    assert bool(torch.isfinite(out.float()).all())
+    rows = np.arange(lq)
+    for h in range(2):
+        ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), 0, h, rows, cos=cos, sin=sin, scale=scale)
+        _check(out, lse, ref, ref_lse, 0, h, rows)
