@@ -8,9 +8,9 @@ blocks; README, "Memory-Efficient Runtime": buffers preallocated from the
 known generation length).  A block can be quantized again in place (the
 streaming runtimes' chunk overwrite, README "Highlights").
 
-This module only sequences library calls (``varq.varq_quantize_pack`` and
-``varq.varq_packed_attention``) and owns the buffers they need; every value is
-computed by the library's kernels.
+This module only sequences library calls (``varq.varq_quantize_pack``,
+``varq.varq_packed_attention`` and ``varq.varq_packed_attention_rope3d``) and
+owns the buffers they need; every value is computed by the library's kernels.
 """
 from __future__ import annotations
 
@@ -60,16 +60,28 @@ class PackedKVLoop:
 
     def attend(self, q: torch.Tensor, n_cached_blocks: int, out: Optional[torch.Tensor] = None,
                lse: Optional[torch.Tensor] = None, rope_cos: Optional[torch.Tensor] = None,
-               rope_sin: Optional[torch.Tensor] = None, softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
-        """Attention of ``q`` (bf16 ``[B, H, lq, D]``) over blocks ``0 .. n_cached_blocks - 1``."""
+               rope_sin: Optional[torch.Tensor] = None, softmax_scale: float = 0.0, stream=None,
+               rope3d: Optional[V.Rope3d] = None) -> torch.Tensor:
+        """Attention of ``q`` (bf16 ``[B, H, lq, D]``) over blocks ``0 .. n_cached_blocks - 1``.
+
+        Pre-RoPE keys: ``rope_cos``/``rope_sin`` tables, or a ``rope3d``
+        schedule whose angles the kernel computes (not both)."""
         if not all(self.cached[:n_cached_blocks]):
             raise RuntimeError("attention over a block that has not been appended")
+        if rope3d is not None and (rope_cos is not None or rope_sin is not None):
+            raise ValueError("pass rope tables or a rope3d schedule, not both")
         if out is None:
             out = torch.empty_like(q)
-        V.varq_packed_attention(self.layout, q, self.k_packed, self.k_meta, self.v_packed, self.v_meta, out,
-                                n_cached_blocks=n_cached_blocks, softmax_scale=softmax_scale,
-                                rope_cos=rope_cos, rope_sin=rope_sin, lse=lse, workspace=self.workspace,
-                                dev_status=self.status, stream=stream)
+        if rope3d is not None:
+            V.varq_packed_attention_rope3d(self.layout, q, self.k_packed, self.k_meta, self.v_packed, self.v_meta,
+                                           out, rope3d, n_cached_blocks=n_cached_blocks,
+                                           softmax_scale=softmax_scale, lse=lse, workspace=self.workspace,
+                                           dev_status=self.status, stream=stream)
+        else:
+            V.varq_packed_attention(self.layout, q, self.k_packed, self.k_meta, self.v_packed, self.v_meta, out,
+                                    n_cached_blocks=n_cached_blocks, softmax_scale=softmax_scale,
+                                    rope_cos=rope_cos, rope_sin=rope_sin, lse=lse, workspace=self.workspace,
+                                    dev_status=self.status, stream=stream)
         return out
 
     def step(self, k: int, k_block: torch.Tensor, v_block: torch.Tensor, q: torch.Tensor,

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 from packed_kv_attention_b200 import synth
+from packed_kv_attention_b200 import varq as V
 from packed_kv_attention_b200.generation import PackedKVLoop
 from test_gpu_attention import DEV, _check, _oracle_attention
 
@@ -133,6 +134,35 @@ def test_generation_loop_next_frame_grouping(frame_tokens):
         lse = torch.empty(B, H, n, dtype=torch.float32, device=DEV)
         out = loop.step(step, kd[:, :, bs[step]:bs[step + 1]], vd[:, :, bs[step]:bs[step + 1]], q.to(DEV), lse=lse,
                         rope_cos=cd, rope_sin=sd)
+        torch.cuda.synchronize()
+        rows = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.integers(0, n, 12)]))
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k, v, q, bs, bits, step + 1, 0, h, rows, cos=cos, sin=sin)
+            _check(out, lse, ref, ref_lse, 0, h, rows)
+    assert loop.device_status() == 0
+
+
+def test_generation_loop_next_frame_schedule():
+    """The next-frame loop with the rotary angles computed in the kernel from
+    the 3D schedule (1,560-token frames on a 52-wide grid): frames appended
+    one at a time, each frame's queries attending to all frames so far,
+    against the oracle rotating by its own restatement of the schedule."""
+    from oracle import varq_oracle as O
+    bits, D, B, H = 3, 128, 1, 2
+    sizes = [1560] * 4
+    g, k, v = _cache(37, B, H, sizes, D)
+    bs = synth.block_starts(sizes)
+    c, s = O.rope_schedule_tables(bs[-1], 1560, 52, synth.rope_axis_pairs(D))
+    cos, sin = torch.from_numpy(c), torch.from_numpy(s)
+    rope = V.Rope3d.make(1560, 52, synth.rope_axis_pairs(D))
+    loop = PackedKVLoop(B, H, D, bits, sizes, device=DEV)
+    kd, vd = k.to(DEV), v.to(DEV)
+    rng = np.random.default_rng(5)
+    for step, n in enumerate(sizes):
+        q = synth.queries(g, B, H, n, D)
+        lse = torch.empty(B, H, n, dtype=torch.float32, device=DEV)
+        out = loop.step(step, kd[:, :, bs[step]:bs[step + 1]], vd[:, :, bs[step]:bs[step + 1]], q.to(DEV), lse=lse,
+                        rope3d=rope)
         torch.cuda.synchronize()
         rows = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.integers(0, n, 12)]))
         for h in range(H):
