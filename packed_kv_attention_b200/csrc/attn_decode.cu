@@ -25,6 +25,7 @@
 // A step across a generation-block boundary looks up each token's own
 // (scale, min) instead of the block constants held in registers.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -40,7 +41,6 @@ constexpr float kDecRescale = 8.0f;  // log2 units
 template <int BITS, int D, int QG>
 struct Dec {
   static constexpr int CPW = 32 / BITS;                // tokens per word
-  static constexpr uint32_t MASK = (1u << BITS) - 1u;
   static constexpr int NCG = D / 16;                   // K: 16-channel groups, one lane each
   static constexpr int LOG_NCG = NCG == 8 ? 3 : 2;
   static constexpr int RPW = 32 / NCG;                 // word rows per warp step
@@ -422,6 +422,347 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __gri
   }
 }
 
+// ---------------------------------------------------------------------------
+// Table form for 2-4-bit codes.  A (block, channel) cell has only 2^b
+// distinct dequantized values bf16(fmaf(code, scale, min)), so the CTA
+// tabulates them in shared memory, K and V, once per generation block, and a
+// code costs a byte permute (its table row offset), one shared load and one
+// fma instead of the arithmetic above.  Tables are [code][channel] fp32 in
+// 64-channel halves of 256-byte rows, so the byte permute that puts the code
+// into byte 1 of an offset yields code * 256 + (channel mod 64) * 4, and the
+// half, the tensor and the table slot are constants folded into the load.
+// Two slots hold consecutive blocks (slot = block & 1); the warps go through
+// their steps in rounds of one step each, and a round that needs a block not
+// yet tabulated rebuilds the slot between two CTA barriers.  A step across a
+// block boundary, or inside a block neither slot holds (rounds spanning more
+// than two blocks), takes the per-token path of the kernel above.
+// K channel map: word i of lane (row r, group cg) holds channel
+// cg + NCG m with m = (i & 8) | ((i + r) & 7) (plus 64 (i >> 3) for D = 128),
+// so in every load the 32 lanes read 32 distinct banks; V lanes own channels
+// lane + 32 k as above, one bank each.
+namespace {
+
+template <int BITS, int D>
+struct Lut {
+  static constexpr int NCODE = 1 << BITS;
+  static constexpr int HALVES = D / 64;
+  static constexpr bool kUsed = BITS <= 4;
+};
+
+// Offsets code * 256 + base (base < 256) of the codes of one packed word.
+// 4- and 2-bit codes: the word is split once into byte planes (plane p holds
+// codes p, p + NP, ... one per byte) and a byte permute places code j's byte
+// into byte 1 of base; 3-bit codes straddle bytes and take a shift and a
+// mask-or each.
+template <int BITS>
+struct CodeOff {
+  static constexpr int NP = BITS == 4 ? 2 : (BITS == 2 ? 4 : 1);
+  uint32_t p[NP];
+  CodeOff() = default;
+  __device__ __forceinline__ explicit CodeOff(uint32_t w) {
+    if constexpr (BITS == 3) {
+      p[0] = w;
+    } else {
+      constexpr uint32_t M = BITS == 4 ? 0x0F0F0F0Fu : 0x03030303u;
+#pragma unroll
+      for (int i = 0; i < NP; ++i) p[i] = (w >> (i * BITS)) & M;
+    }
+  }
+  __device__ __forceinline__ uint32_t at(int j, uint32_t base) const {
+    if constexpr (BITS == 3) {
+      const int o = 3 * j;
+      const uint32_t x = o >= 8 ? (p[0] >> (o - 8)) : (p[0] << (8 - o));
+      return (x & 0x700u) | base;
+    } else {
+      return __byte_perm(p[j % NP], base, 0x7604u | (uint32_t(j / NP) << 4));
+    }
+  }
+};
+
+// Entry at byte offset off of half h of table (slot S, tensor T); with S and T
+// template arguments and h known once the loops are unrolled, all but off is
+// an immediate of the shared load.
+template <int S, int T, int NCODE, int HALVES>
+__device__ __forceinline__ float lut_at(const float (&tbl)[2][2][HALVES][NCODE][64], int h, uint32_t off) {
+  return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(&tbl[S][T][h][0][0]) + off);
+}
+
+}  // namespace
+
+template <int BITS, int D>
+__global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const __grid_constant__ AttnArgs a) {
+  using C = Dec<BITS, D, 1>;
+  using TB = Lut<BITS, D>;
+  constexpr int CPW = C::CPW, NCG = C::NCG, RPW = C::RPW, TPS = C::TPS, CPL = C::CPL;
+  constexpr int NV = C::NV, NVP = C::NVP, VPL = C::VPL;
+  constexpr int NCODE = TB::NCODE, HALVES = TB::HALVES;
+  __shared__ int sm_bs[VARQ_MAX_BLOCKS + 1];
+  __shared__ float sm_q[D];
+  __shared__ float sm_p[kDecWarps][TPS];
+  __shared__ float sm_o[kDecWarps][D];
+  __shared__ float sm_ml[kDecWarps][2];
+  __shared__ __align__(16) float sm_lut[2][2][HALVES][NCODE][64];  // [slot][K, V][half][code][channel % 64]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x % a.lq, split = blockIdx.x / a.lq;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = int64_t(b) * a.heads + h;
+  const float sl2 = a.scale_log2;
+  const int ncb = a.n_cached_blocks;
+
+  for (int i = tid; i <= ncb; i += kDecThreads) sm_bs[i] = a.block_start[i];
+  for (int d = tid; d < D; d += kDecThreads)
+    sm_q[d] = __bfloat162float(a.q[int64_t(b) * a.q_sb + int64_t(h) * a.q_sh + int64_t(row) * a.q_st + d]);
+  __syncthreads();
+
+  // this CTA's word rows [w_begin, w_end), as in the kernel above
+  const int t_att = a.t_att;
+  const int words_att = (t_att + CPW - 1) / CPW;
+  const int per = ((words_att + a.n_splits - 1) / a.n_splits + RPW - 1) / RPW * RPW;
+  const int w_begin = min(words_att, split * per), w_end = min(words_att, w_begin + per);
+  const int nsteps = (w_end - w_begin + RPW - 1) / RPW;
+
+  const int r = lane / NCG, cg = lane % NCG;
+  const uint32_t* kw_base = a.k_packed + bh * a.words_per_row * D;
+  const uint32_t* vw_base = a.v_packed + bh * a.words_per_row * D;
+  const uint32_t* km_base = a.k_meta + bh * a.n_blocks_total * D;
+  const uint32_t* vm_base = a.v_meta + bh * a.n_blocks_total * D;
+
+  // K: channel of word i and its byte offset within a 64-channel table row
+  auto kchan = [&](int i) {
+    const int m = (i & 8) | ((i + r) & 7);
+    return D == 128 ? 64 * (i >> 3) + cg + 8 * (m & 7) : cg + 4 * m;
+  };
+  float qs[16];
+  uint32_t bk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = kchan(i);
+    qs[i] = sm_q[c] * sl2;
+    bk[i] = uint32_t(c & 63) * 4u;
+  }
+  uint32_t bv[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) bv[k] = uint32_t((lane + 32 * k) & 63) * 4u;
+
+  // tabulate block blk into slot blk & 1: one (tensor, channel) per thread,
+  // the K or V value of every code
+  auto build = [&](int blk) {
+    const int sl = blk & 1;
+    for (int e = tid; e < 2 * D; e += kDecThreads) {
+      const int t = e / D, c = e - t * D;
+      const float2 sm = meta_unpack(__ldg((t ? vm_base : km_base) + int64_t(blk) * D + c));
+#pragma unroll
+      for (int code = 0; code < NCODE; ++code)
+        sm_lut[sl][t][c >> 6][code][c & 63] = bf16_round(__fmaf_rn(float(code), sm.x, sm.y));
+    }
+  };
+
+  float m_run = -__int_as_float(0x7F800000), l_run = 0.0f, O[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) O[k] = 0.0f;
+
+  int held0 = -1, held1 = -1;  // block tabulated in slot 0 / slot 1
+  int bq = 0;                  // block of the round's first token
+  const int nrounds = (nsteps + kDecWarps - 1) / kDecWarps;
+  for (int rd = 0; rd < nrounds; ++rd) {
+    // ---- the blocks this round reaches: the first and (if reached) the next
+    const int s0 = rd * kDecWarps;
+    const int rts = (w_begin + s0 * RPW) * CPW;
+    const int rte = min(min(w_begin + (s0 + kDecWarps) * RPW, w_end) * CPW, t_att);
+    while (bq + 1 < ncb && rts >= sm_bs[bq + 1]) ++bq;
+    const bool two = bq + 1 < ncb && rte > sm_bs[bq + 1];
+    const bool need_a = ((bq & 1) ? held1 : held0) != bq;
+    const bool need_b = two && (((bq + 1) & 1) ? held1 : held0) != bq + 1;
+    if (need_a || need_b) {  // uniform over the CTA
+      __syncthreads();       // no warp still reads the slots of the last round
+      if (need_a) build(bq);
+      if (need_b) build(bq + 1);
+      __syncthreads();
+      if (need_a) (bq & 1 ? held1 : held0) = bq;
+      if (need_b) ((bq + 1) & 1 ? held1 : held0) = bq + 1;
+    }
+
+    const int s = s0 + warp;
+    if (s >= nsteps) continue;
+    const int wr0 = w_begin + s * RPW;
+    const int ts = wr0 * CPW;
+    const int te = min(min(wr0 + RPW, w_end) * CPW, t_att);
+    const int wk = wr0 + r;
+    const int tr = wk * CPW;
+    int blk = bq;
+    while (blk + 1 < ncb && ts >= sm_bs[blk + 1]) ++blk;
+    const bool across = blk + 1 < ncb && te > sm_bs[blk + 1];
+    // 0 / 1: the step lies in the block slot 0 / 1 holds; 2: per-token path
+    const int mode = across ? 2 : (held0 == blk ? 0 : (held1 == blk ? 1 : 2));
+
+    uint32_t kw[16], vw[RPW][CPL];
+    if (mode < 2) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) kw[i] = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + kchan(i)) : 0u;
+    }
+    constexpr bool kEarlyV = NVP <= 8;
+    auto load_v = [&]() {
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+          vw[rr][k] = wr0 + rr < w_end ? __ldg(vw_base + int64_t(wr0 + rr) * D + lane + 32 * k) : 0u;
+    };
+    if (kEarlyV) load_v();
+
+    // ---- scores of the lane's row over its 16 channels, summed over the row's lanes
+    float acc[NVP];
+#pragma unroll
+    for (int i = 0; i < NVP; ++i) acc[i] = 0.0f;
+    auto scores_tab = [&](auto slot) {
+      constexpr int S = decltype(slot)::value;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const CodeOff<BITS> co(kw[i]);
+#pragma unroll
+        for (int j = 0; j < CPW; ++j)
+          acc[j] = __fmaf_rn(qs[i], lut_at<S, 0>(sm_lut, D == 128 ? (i >> 3) : 0, co.at(j, bk[i])), acc[j]);
+      }
+    };
+    if (mode == 0) {
+      scores_tab(std::integral_constant<int, 0>{});
+    } else if (mode == 1) {
+      scores_tab(std::integral_constant<int, 1>{});
+    } else {
+      int tb[CPW];  // block of each token of the lane's row
+      {
+        int bb = blk;
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          while (bb + 1 < ncb && tr + j >= sm_bs[bb + 1]) ++bb;
+          tb[j] = bb;
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t w = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + cg * 16 + c) : 0u;
+        const float qv = sm_q[cg * 16 + c] * sl2;
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const float2 sm = meta_unpack(__ldg(km_base + int64_t(tb[j]) * D + cg * 16 + c));
+          acc[j] = __fmaf_rn(qv, bf16_round(__fmaf_rn(code_f<BITS>(w, j), sm.x, sm.y)), acc[j]);
+        }
+      }
+    }
+    reduce_scatter<NVP, C::LOG_NCG>(acc, lane);
+
+    // ---- online softmax over this step (the kernel above with one row)
+    const int idx0 = VPL * bitrev<C::LOG_NCG>(cg);
+    {
+      float mx = -__int_as_float(0x7F800000);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV && tr + idx < te) mx = fmaxf(mx, acc[i]);
+      }
+      if (__any_sync(0xFFFFFFFFu, mx > m_run + kDecRescale)) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = ex2_approx(m_run - mn);
+        l_run *= alpha;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) O[k] *= alpha;
+        m_run = mn;
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV) {
+          const float p = tr + idx < te ? ex2_approx(acc[i] - m_run) : 0.0f;
+          l_run += p;
+          sm_p[warp][r * CPW + idx] = p;
+        }
+      }
+    }
+    __syncwarp();
+    if (!kEarlyV) load_v();
+
+    // ---- O += P V_hat; tokens past the range have P = 0
+    auto pv_tab = [&](auto slot) {
+      constexpr int S = decltype(slot)::value;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+        CodeOff<BITS> co[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) co[k] = CodeOff<BITS>(vw[rr][k]);
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const float p = sm_p[warp][rr * CPW + j];
+#pragma unroll
+          for (int k = 0; k < CPL; ++k)
+            O[k] = __fmaf_rn(p, lut_at<S, 1>(sm_lut, k >> 1, co[k].at(j, bv[k])), O[k]);
+        }
+      }
+    };
+    if (mode == 0) {
+      pv_tab(std::integral_constant<int, 0>{});
+    } else if (mode == 1) {
+      pv_tab(std::integral_constant<int, 1>{});
+    } else {
+      int bb = blk;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const int t = ts + rr * CPW + j;
+          while (bb + 1 < ncb && t >= sm_bs[bb + 1]) ++bb;
+          const float p = sm_p[warp][rr * CPW + j];
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const float2 sm = meta_unpack(__ldg(vm_base + int64_t(bb) * D + lane + 32 * k));
+            O[k] = __fmaf_rn(p, bf16_round(__fmaf_rn(code_f<BITS>(vw[rr][k], j), sm.x, sm.y)), O[k]);
+          }
+        }
+      }
+    }
+    __syncwarp();  // sm_p is rewritten by the next step
+  }
+
+  // ---- merge the warps' (m, l, O) into this range's partial
+  {
+    float ls = l_run;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o);
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) sm_o[warp][lane + 32 * k] = O[k];
+    if (lane == 0) {
+      sm_ml[warp][0] = m_run;
+      sm_ml[warp][1] = ls;
+    }
+  }
+  __syncthreads();
+  for (int d = tid; d < D; d += kDecThreads) {
+    float M = -__int_as_float(0x7F800000);
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_ml[w][0]);
+    float o = 0.0f, L = 0.0f;
+    if (M != -__int_as_float(0x7F800000)) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mw = sm_ml[w][0];
+        if (mw == -__int_as_float(0x7F800000)) continue;
+        const float f = ex2_approx(mw - M);
+        o = __fmaf_rn(f, sm_o[w][d], o);
+        L = __fmaf_rn(f, sm_ml[w][1], L);
+      }
+    }
+    float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
+                int64_t(row) * (D + 2);
+    ws[d] = o;
+    if (d == 0) {
+      ws[D] = M;
+      ws[D + 1] = L;
+    }
+  }
+}
+
 namespace {
 
 // Query rows per CTA (more rows run as more row groups over the same range).
@@ -437,10 +778,25 @@ cudaError_t launch_dec(const AttnArgs& a, cudaStream_t stream) {
   return launch_attention_combine(a, stream);
 }
 
+template <int BITS, int D>
+cudaError_t launch_dec_lut(const AttnArgs& a, cudaStream_t stream) {
+  const dim3 grid(unsigned(a.lq * a.n_splits), unsigned(a.heads), unsigned(a.batch));
+  attn_decode_lut_kernel<BITS, D><<<grid, kDecThreads, 0, stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attention_combine(a, stream);
+}
+
+// 2-4-bit codes: the table form; wider codes: the arithmetic form.
 template <int BITS>
 cudaError_t launch_dec_bits(const AttnArgs& a, cudaStream_t s) {
-  if (a.head_dim == 128) return launch_dec<BITS, 128, kDecQG>(a, s);
-  if (a.head_dim == 64) return launch_dec<BITS, 64, kDecQG>(a, s);
+  if constexpr (Lut<BITS, 128>::kUsed) {
+    if (a.head_dim == 128) return launch_dec_lut<BITS, 128>(a, s);
+    if (a.head_dim == 64) return launch_dec_lut<BITS, 64>(a, s);
+  } else {
+    if (a.head_dim == 128) return launch_dec<BITS, 128, kDecQG>(a, s);
+    if (a.head_dim == 64) return launch_dec<BITS, 64, kDecQG>(a, s);
+  }
   return cudaErrorInvalidValue;
 }
 

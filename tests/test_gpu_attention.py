@@ -216,6 +216,26 @@ def test_attention_decode_from_codes(bits, D, lq):
             _check(out, lse, ref, ref_lse, b, h, rows)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_decode_block_tables(bits, D):
+    """Split-KV form for one and two query rows with 2-4-bit codes, which the
+    kernel dequantizes through per-block value tables: blocks of 33-700 tokens,
+    so the tables are rebuilt as each KV range moves on and its rounds of
+    steps reach one, two or three blocks."""
+    B, H = 1, 3
+    sizes = [700, 90, 130, 257, 64, 129, 33, 520, 300]
+    bs = synth.block_starts(sizes)
+    for lq in (1, 2):
+        k, v, q, _, _ = _inputs(B, H, D, sizes, lq, seed=bits * 7 + D + lq)
+        L = V.varq_cache_alloc(B, H, D, bits, bs)
+        out, lse = _gpu_attention(L, k, v, q, len(sizes), path=V.PATH_SPLIT)
+        rows = np.arange(lq)
+        for h in range(H):
+            ref, ref_lse = _oracle_attention(k, v, q, bs, bits, len(sizes), 0, h, rows)
+            _check(out, lse, ref, ref_lse, 0, h, rows)
+
+
 def _spiked_inputs(B, H, D, T, lq, spikes, seed):
     """Keys and values ~ N(0, 1), queries sharing a direction u; token t of
     every (b, h) gets key beta * u for each (t, beta) in spikes, so its score
