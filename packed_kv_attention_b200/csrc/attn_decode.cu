@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
   constexpr int NCODE = TB::NCODE, HALVES = TB::HALVES;
   __shared__ int sm_bs[VARQ_MAX_BLOCKS + 1];
   __shared__ float sm_q[D];
-  __shared__ float sm_p[kDecWarps][TPS];
+  __shared__ __align__(16) float sm_p[kDecWarps][TPS];
   __shared__ float sm_o[kDecWarps][D];
   __shared__ float sm_ml[kDecWarps][2];
   __shared__ __align__(16) float sm_lut[2][2][HALVES][NCODE][64];  // [slot][K, V][half][code][channel % 64]
@@ -692,12 +692,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
         CodeOff<BITS> co[CPL];
 #pragma unroll
         for (int k = 0; k < CPL; ++k) co[k] = CodeOff<BITS>(vw[rr][k]);
+        constexpr int PV = CPW % 4 == 0 ? 4 : 2;  // P values per shared load
 #pragma unroll
-        for (int j = 0; j < CPW; ++j) {
-          const float p = sm_p[warp][rr * CPW + j];
+        for (int j0 = 0; j0 < CPW; j0 += PV) {
+          float pj[PV];
+          if constexpr (PV == 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(&sm_p[warp][rr * CPW + j0]);
+            pj[0] = t4.x; pj[1] = t4.y; pj[2] = t4.z; pj[3] = t4.w;
+          } else {
+            const float2 t2 = *reinterpret_cast<const float2*>(&sm_p[warp][rr * CPW + j0]);
+            pj[0] = t2.x; pj[1] = t2.y;
+          }
 #pragma unroll
-          for (int k = 0; k < CPL; ++k)
-            O[k] = __fmaf_rn(p, lut_at<S, 1>(sm_lut, k >> 1, co[k].at(j, bv[k])), O[k]);
+          for (int u = 0; u < PV; ++u)
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+              O[k] = __fmaf_rn(pj[u], lut_at<S, 1>(sm_lut, k >> 1, co[k].at(j0 + u, bv[k])), O[k]);
         }
       }
     };
