@@ -446,7 +446,6 @@ template <int BITS, int D>
 struct Lut {
   static constexpr int NCODE = 1 << BITS;
   static constexpr int HALVES = D / 64;
-  static constexpr bool kUsed = BITS <= 4;
 };
 
 // Offsets code * 256 + base (base < 256) of the codes of one packed word.
@@ -533,34 +532,41 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
     const int m = (i & 8) | ((i + r) & 7);
     return D == 128 ? 64 * (i >> 3) + cg + 8 * (m & 7) : cg + 4 * m;
   };
-  float qs[16];
   uint32_t bk[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int c = kchan(i);
-    qs[i] = sm_q[c] * sl2;
-    bk[i] = uint32_t(c & 63) * 4u;
-  }
+  for (int i = 0; i < 16; ++i) bk[i] = uint32_t(kchan(i) & 63) * 4u;
   uint32_t bv[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) bv[k] = uint32_t((lane + 32 * k) & 63) * 4u;
 
   // tabulate block blk into slot blk & 1: one (tensor, channel) per thread,
-  // the K or V value of every code
+  // for every code the V value and the K value times the query channel
+  // (pre-scaled by scale log2 e), so a score is a sum of table entries
   auto build = [&](int blk) {
     const int sl = blk & 1;
     for (int e = tid; e < 2 * D; e += kDecThreads) {
       const int t = e / D, c = e - t * D;
       const float2 sm = meta_unpack(__ldg((t ? vm_base : km_base) + int64_t(blk) * D + c));
+      const float qc = t ? 1.0f : sm_q[c] * sl2;
 #pragma unroll
       for (int code = 0; code < NCODE; ++code)
-        sm_lut[sl][t][c >> 6][code][c & 63] = bf16_round(__fmaf_rn(float(code), sm.x, sm.y));
+        sm_lut[sl][t][c >> 6][code][c & 63] = qc * bf16_round(__fmaf_rn(float(code), sm.x, sm.y));
     }
   };
 
   float m_run = -__int_as_float(0x7F800000), l_run = 0.0f, O[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) O[k] = 0.0f;
+
+  // K words of a step in the table form's channel map (zero past the range)
+  uint32_t kw_next[16];
+  auto load_k = [&](int st) {
+    const int wk = w_begin + st * RPW + r;
+    const bool in = st < nsteps && wk < w_end;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) kw_next[i] = in ? __ldg(kw_base + int64_t(wk) * D + kchan(i)) : 0u;
+  };
+  load_k(warp);
 
   int held0 = -1, held1 = -1;  // block tabulated in slot 0 / slot 1
   int bq = 0;                  // block of the round's first token
@@ -596,11 +602,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
     // 0 / 1: the step lies in the block slot 0 / 1 holds; 2: per-token path
     const int mode = across ? 2 : (held0 == blk ? 0 : (held1 == blk ? 1 : 2));
 
+    // this step's K words (loaded one step ahead); then the next step's
     uint32_t kw[16], vw[RPW][CPL];
-    if (mode < 2) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) kw[i] = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + kchan(i)) : 0u;
-    }
+    for (int i = 0; i < 16; ++i) kw[i] = kw_next[i];
+    load_k(s + kDecWarps);
     constexpr bool kEarlyV = NVP <= 8;
     auto load_v = [&]() {
 #pragma unroll
@@ -622,7 +628,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
         const CodeOff<BITS> co(kw[i]);
 #pragma unroll
         for (int j = 0; j < CPW; ++j)
-          acc[j] = __fmaf_rn(qs[i], lut_at<S, 0>(sm_lut, D == 128 ? (i >> 3) : 0, co.at(j, bk[i])), acc[j]);
+          acc[j] = __fadd_rn(acc[j], lut_at<S, 0>(sm_lut, D == 128 ? (i >> 3) : 0, co.at(j, bk[i])));
       }
     };
     if (mode == 0) {
@@ -800,7 +806,7 @@ cudaError_t launch_dec_lut(const AttnArgs& a, cudaStream_t stream) {
 // 2-4-bit codes: the table form; wider codes: the arithmetic form.
 template <int BITS>
 cudaError_t launch_dec_bits(const AttnArgs& a, cudaStream_t s) {
-  if constexpr (Lut<BITS, 128>::kUsed) {
+  if constexpr (BITS <= 4) {
     if (a.head_dim == 128) return launch_dec_lut<BITS, 128>(a, s);
     if (a.head_dim == 64) return launch_dec_lut<BITS, 64>(a, s);
   } else {
