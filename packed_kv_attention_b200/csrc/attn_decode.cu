@@ -432,9 +432,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __gri
 // into byte 1 of an offset yields code * 256 + (channel mod 64) * 4, and the
 // half, the tensor and the table slot are constants folded into the load.
 // Two slots hold consecutive blocks (slot = block & 1); the warps go through
-// their steps in rounds of one step each, and a round that needs a block not
+// their steps in waves of one step each, and a wave that needs a block not
 // yet tabulated rebuilds the slot between two CTA barriers.  A step across a
-// block boundary, or inside a block neither slot holds (rounds spanning more
+// block boundary, or inside a block neither slot holds (waves spanning more
 // than two blocks), takes the per-token path of the kernel above.
 // K channel map: word i of lane (row r, group cg) holds channel
 // cg + NCG m with m = (i & 8) | ((i + r) & 7) (plus 64 (i >> 3) for D = 128),
@@ -569,11 +569,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
   load_k(warp);
 
   int held0 = -1, held1 = -1;  // block tabulated in slot 0 / slot 1
-  int bq = 0;                  // block of the round's first token
-  const int nrounds = (nsteps + kDecWarps - 1) / kDecWarps;
-  for (int rd = 0; rd < nrounds; ++rd) {
-    // ---- the blocks this round reaches: the first and (if reached) the next
-    const int s0 = rd * kDecWarps;
+  int bq = 0;                  // block of the wave's first token
+  const int nwaves = (nsteps + kDecWarps - 1) / kDecWarps;
+  for (int wv = 0; wv < nwaves; ++wv) {
+    // ---- the blocks this wave reaches: the first and (if reached) the next
+    const int s0 = wv * kDecWarps;
     const int rts = (w_begin + s0 * RPW) * CPW;
     const int rte = min(min(w_begin + (s0 + kDecWarps) * RPW, w_end) * CPW, t_att);
     while (bq + 1 < ncb && rts >= sm_bs[bq + 1]) ++bq;
@@ -581,7 +581,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
     const bool need_a = ((bq & 1) ? held1 : held0) != bq;
     const bool need_b = two && (((bq + 1) & 1) ? held1 : held0) != bq + 1;
     if (need_a || need_b) {  // uniform over the CTA
-      __syncthreads();       // no warp still reads the slots of the last round
+      __syncthreads();       // no warp still reads the slots of the last wave
       if (need_a) build(bq);
       if (need_b) build(bq + 1);
       __syncthreads();

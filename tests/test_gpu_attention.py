@@ -221,7 +221,7 @@ def test_attention_decode_from_codes(bits, D, lq):
 def test_attention_decode_block_tables(bits, D):
     """Split-KV form for one and two query rows with 2-4-bit codes, which the
     kernel dequantizes through per-block value tables: blocks of 33-700 tokens,
-    so the tables are rebuilt as each KV range moves on and its rounds of
+    so the tables are rebuilt as each KV range moves on and its waves of
     steps reach one, two or three blocks."""
     B, H = 1, 3
     sizes = [700, 90, 130, 257, 64, 129, 33, 520, 300]
