@@ -26,6 +26,7 @@
 // (scale, min) instead of the block constants held in registers.
 #include <algorithm>
 #include <type_traits>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -486,6 +487,35 @@ __device__ __forceinline__ float lut_at(const float (&tbl)[2][2][HALVES][NCODE][
   return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(&tbl[S][T][h][0][0]) + off);
 }
 
+// f(integral_constant<int, g>) for g = 0 .. QG-1: the row index a compile-time
+// constant, so per-row state stays in registers.
+template <typename F, int... G>
+__device__ __forceinline__ void for_each_row(F&& f, std::integer_sequence<int, G...>) {
+  (f(std::integral_constant<int, G>{}), ...);
+}
+
+// QG consecutive fp32 values of shared memory (16- or 8-byte aligned) in one load.
+template <int QG>
+struct RowVals {
+  float v[QG];
+};
+template <int QG>
+__device__ __forceinline__ RowVals<QG> rows_load(const float* p) {
+  RowVals<QG> r;
+  if constexpr (QG == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    r.v[0] = t.x;
+    r.v[1] = t.y;
+    r.v[2] = t.z;
+    r.v[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    r.v[0] = t.x;
+    r.v[1] = t.y;
+  }
+  return r;
+}
+
 }  // namespace
 
 template <int BITS, int D>
@@ -779,10 +809,312 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_kernel(const _
   }
 }
 
+// The table form for 2 to 4 query rows per CTA: each dequantized code serves
+// every row.  The K table holds the values themselves (a row-independent
+// table) and each code feeds QG fmas, the rows' query channels coming from
+// shared memory with one vector load per packed word; P of a token for all
+// rows comes the same way.  Otherwise as the kernel above (no K prefetch: the
+// registers go to the QG rows' partial scores).
+template <int BITS, int D, int QG>
+__global__ void __launch_bounds__(kDecThreads, 2) attn_decode_lut_rows_kernel(const __grid_constant__ AttnArgs a) {
+  using C = Dec<BITS, D, QG>;
+  using TB = Lut<BITS, D>;
+  constexpr int CPW = C::CPW, NCG = C::NCG, RPW = C::RPW, TPS = C::TPS, CPL = C::CPL;
+  constexpr int NV = C::NV, NVP = C::NVP, VPL = C::VPL;
+  constexpr int NCODE = TB::NCODE, HALVES = TB::HALVES;
+  static_assert(QG == 2 || QG == 4, "rows per CTA");
+  __shared__ int sm_bs[VARQ_MAX_BLOCKS + 1];
+  __shared__ __align__(16) float sm_q[D][QG];                      // pre-scaled by scale log2 e
+  __shared__ __align__(16) float sm_p[kDecWarps][TPS][QG];
+  __shared__ float sm_ml[kDecWarps][QG][2];
+  __shared__ __align__(16) float sm_lut[2][2][HALVES][NCODE][64];  // [slot][K, V][half][code][channel % 64]
+  // per-warp O for the merge, in the table storage once every step is done
+  static_assert(sizeof(float) * kDecWarps * QG * D <= sizeof(sm_lut), "merge buffer");
+  float(*sm_o)[QG][D] = reinterpret_cast<float(*)[QG][D]>(&sm_lut[0][0][0][0][0]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nrg = (a.lq + QG - 1) / QG;
+  const int rg = blockIdx.x % nrg, split = blockIdx.x / nrg;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = int64_t(b) * a.heads + h;
+  const float sl2 = a.scale_log2;
+  const int ncb = a.n_cached_blocks;
+
+  for (int i = tid; i <= ncb; i += kDecThreads) sm_bs[i] = a.block_start[i];
+  for (int i = tid; i < QG * D; i += kDecThreads) {
+    const int g = i / D, d = i % D, row = rg * QG + g;
+    sm_q[d][g] = row < a.lq ? __bfloat162float(a.q[int64_t(b) * a.q_sb + int64_t(h) * a.q_sh + int64_t(row) * a.q_st + d]) * sl2
+                            : 0.0f;
+  }
+  __syncthreads();
+
+  const int t_att = a.t_att;
+  const int words_att = (t_att + CPW - 1) / CPW;
+  const int per = ((words_att + a.n_splits - 1) / a.n_splits + RPW - 1) / RPW * RPW;
+  const int w_begin = min(words_att, split * per), w_end = min(words_att, w_begin + per);
+  const int nsteps = (w_end - w_begin + RPW - 1) / RPW;
+
+  const int r = lane / NCG, cg = lane % NCG;
+  const uint32_t* kw_base = a.k_packed + bh * a.words_per_row * D;
+  const uint32_t* vw_base = a.v_packed + bh * a.words_per_row * D;
+  const uint32_t* km_base = a.k_meta + bh * a.n_blocks_total * D;
+  const uint32_t* vm_base = a.v_meta + bh * a.n_blocks_total * D;
+
+  auto kchan = [&](int i) {
+    const int m = (i & 8) | ((i + r) & 7);
+    return D == 128 ? 64 * (i >> 3) + cg + 8 * (m & 7) : cg + 4 * m;
+  };
+  uint32_t bk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) bk[i] = uint32_t(kchan(i) & 63) * 4u;
+  uint32_t bv[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) bv[k] = uint32_t((lane + 32 * k) & 63) * 4u;
+
+  // tabulate block blk into slot blk & 1: the K and V values of every code
+  auto build = [&](int blk) {
+    const int sl = blk & 1;
+    for (int e = tid; e < 2 * D; e += kDecThreads) {
+      const int t = e / D, c = e - t * D;
+      const float2 sm = meta_unpack(__ldg((t ? vm_base : km_base) + int64_t(blk) * D + c));
+#pragma unroll
+      for (int code = 0; code < NCODE; ++code)
+        sm_lut[sl][t][c >> 6][code][c & 63] = bf16_round(__fmaf_rn(float(code), sm.x, sm.y));
+    }
+  };
+
+  float m_run[QG], l_run[QG], O[QG][CPL];
+#pragma unroll
+  for (int g = 0; g < QG; ++g) {
+    m_run[g] = -__int_as_float(0x7F800000);
+    l_run[g] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) O[g][k] = 0.0f;
+  }
+
+  int held0 = -1, held1 = -1;  // block tabulated in slot 0 / slot 1
+  int bq = 0;                  // block of the wave's first token
+  const int nwaves = (nsteps + kDecWarps - 1) / kDecWarps;
+  for (int wv = 0; wv < nwaves; ++wv) {
+    const int s0 = wv * kDecWarps;
+    const int rts = (w_begin + s0 * RPW) * CPW;
+    const int rte = min(min(w_begin + (s0 + kDecWarps) * RPW, w_end) * CPW, t_att);
+    while (bq + 1 < ncb && rts >= sm_bs[bq + 1]) ++bq;
+    const bool two = bq + 1 < ncb && rte > sm_bs[bq + 1];
+    const bool need_a = ((bq & 1) ? held1 : held0) != bq;
+    const bool need_b = two && (((bq + 1) & 1) ? held1 : held0) != bq + 1;
+    if (need_a || need_b) {  // uniform over the CTA
+      __syncthreads();
+      if (need_a) build(bq);
+      if (need_b) build(bq + 1);
+      __syncthreads();
+      if (need_a) (bq & 1 ? held1 : held0) = bq;
+      if (need_b) ((bq + 1) & 1 ? held1 : held0) = bq + 1;
+    }
+
+    const int s = s0 + warp;
+    if (s >= nsteps) continue;
+    const int wr0 = w_begin + s * RPW;
+    const int ts = wr0 * CPW;
+    const int te = min(min(wr0 + RPW, w_end) * CPW, t_att);
+    const int wk = wr0 + r;
+    const int tr = wk * CPW;
+    int blk = bq;
+    while (blk + 1 < ncb && ts >= sm_bs[blk + 1]) ++blk;
+    const bool across = blk + 1 < ncb && te > sm_bs[blk + 1];
+    const int mode = across ? 2 : (held0 == blk ? 0 : (held1 == blk ? 1 : 2));
+
+    uint32_t kw[16], vw[RPW][CPL];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) kw[i] = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + kchan(i)) : 0u;
+
+    // ---- partial scores acc[g * CPW + j]: row g, token tr + j, the lane's 16 channels
+    float acc[NVP];
+#pragma unroll
+    for (int i = 0; i < NVP; ++i) acc[i] = 0.0f;
+    auto scores_tab = [&](auto slot) {
+      constexpr int S = decltype(slot)::value;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const RowVals<QG> qv = rows_load<QG>(&sm_q[kchan(i)][0]);
+        const CodeOff<BITS> co(kw[i]);
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const float x = lut_at<S, 0>(sm_lut, D == 128 ? (i >> 3) : 0, co.at(j, bk[i]));
+#pragma unroll
+          for (int g = 0; g < QG; ++g) acc[g * CPW + j] = __fmaf_rn(qv.v[g], x, acc[g * CPW + j]);
+        }
+      }
+    };
+    if (mode == 0) {
+      scores_tab(std::integral_constant<int, 0>{});
+    } else if (mode == 1) {
+      scores_tab(std::integral_constant<int, 1>{});
+    } else {
+      int tb[CPW];
+      {
+        int bb = blk;
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          while (bb + 1 < ncb && tr + j >= sm_bs[bb + 1]) ++bb;
+          tb[j] = bb;
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t w = wk < w_end ? __ldg(kw_base + int64_t(wk) * D + cg * 16 + c) : 0u;
+        const RowVals<QG> qv = rows_load<QG>(&sm_q[cg * 16 + c][0]);
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const float2 sm = meta_unpack(__ldg(km_base + int64_t(tb[j]) * D + cg * 16 + c));
+          const float x = bf16_round(__fmaf_rn(code_f<BITS>(w, j), sm.x, sm.y));
+#pragma unroll
+          for (int g = 0; g < QG; ++g) acc[g * CPW + j] = __fmaf_rn(qv.v[g], x, acc[g * CPW + j]);
+        }
+      }
+    }
+    reduce_scatter<NVP, C::LOG_NCG>(acc, lane);
+
+    // ---- online softmax per row over this step; the lane's VPL scores are
+    // partials idx = VPL bitrev(cg) + i: row idx / CPW, token tr + idx % CPW
+    const int idx0 = VPL * bitrev<C::LOG_NCG>(cg);
+    auto softmax_row = [&](auto row_c) {
+      constexpr int g = decltype(row_c)::value;
+      float mx = -__int_as_float(0x7F800000);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV && idx / CPW == g && tr + idx % CPW < te) mx = fmaxf(mx, acc[i]);
+      }
+      if (__any_sync(0xFFFFFFFFu, mx > m_run[g] + kDecRescale)) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        const float mn = fmaxf(m_run[g], mx);
+        const float alpha = ex2_approx(m_run[g] - mn);
+        l_run[g] *= alpha;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) O[g][k] *= alpha;
+        m_run[g] = mn;
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int idx = idx0 + i;
+        if (idx < NV && idx / CPW == g) {
+          const int j = idx % CPW;
+          const float p = tr + j < te ? ex2_approx(acc[i] - m_run[g]) : 0.0f;
+          l_run[g] += p;
+          sm_p[warp][r * CPW + j][g] = p;
+        }
+      }
+    };
+    for_each_row(softmax_row, std::make_integer_sequence<int, QG>{});
+    __syncwarp();
+#pragma unroll
+    for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+      for (int k = 0; k < CPL; ++k)
+        vw[rr][k] = wr0 + rr < w_end ? __ldg(vw_base + int64_t(wr0 + rr) * D + lane + 32 * k) : 0u;
+
+    // ---- O += P V_hat for every row; tokens past the range have P = 0
+    auto pv_tab = [&](auto slot) {
+      constexpr int S = decltype(slot)::value;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+        CodeOff<BITS> co[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) co[k] = CodeOff<BITS>(vw[rr][k]);
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const RowVals<QG> pg = rows_load<QG>(&sm_p[warp][rr * CPW + j][0]);
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const float x = lut_at<S, 1>(sm_lut, k >> 1, co[k].at(j, bv[k]));
+#pragma unroll
+            for (int g = 0; g < QG; ++g) O[g][k] = __fmaf_rn(pg.v[g], x, O[g][k]);
+          }
+        }
+      }
+    };
+    if (mode == 0) {
+      pv_tab(std::integral_constant<int, 0>{});
+    } else if (mode == 1) {
+      pv_tab(std::integral_constant<int, 1>{});
+    } else {
+      int bb = blk;
+#pragma unroll
+      for (int rr = 0; rr < RPW; ++rr) {
+#pragma unroll
+        for (int j = 0; j < CPW; ++j) {
+          const int t = ts + rr * CPW + j;
+          while (bb + 1 < ncb && t >= sm_bs[bb + 1]) ++bb;
+          const RowVals<QG> pg = rows_load<QG>(&sm_p[warp][rr * CPW + j][0]);
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const float2 sm = meta_unpack(__ldg(vm_base + int64_t(bb) * D + lane + 32 * k));
+            const float x = bf16_round(__fmaf_rn(code_f<BITS>(vw[rr][k], j), sm.x, sm.y));
+#pragma unroll
+            for (int g = 0; g < QG; ++g) O[g][k] = __fmaf_rn(pg.v[g], x, O[g][k]);
+          }
+        }
+      }
+    }
+    __syncwarp();  // sm_p is rewritten by the next step
+  }
+
+  // ---- merge the warps' (m, l, O) into this range's partial, per row
+  __syncthreads();  // every warp is done with the tables, which now hold O
+#pragma unroll
+  for (int g = 0; g < QG; ++g) {
+    float ls = l_run[g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, o);
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) sm_o[warp][g][lane + 32 * k] = O[g][k];
+    if (lane == 0) {
+      sm_ml[warp][g][0] = m_run[g];
+      sm_ml[warp][g][1] = ls;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < QG * D; i += kDecThreads) {
+    const int g = i / D, d = i % D, row = rg * QG + g;
+    if (row >= a.lq) continue;
+    float M = -__int_as_float(0x7F800000);
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_ml[w][g][0]);
+    float o = 0.0f, L = 0.0f;
+    if (M != -__int_as_float(0x7F800000)) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mw = sm_ml[w][g][0];
+        if (mw == -__int_as_float(0x7F800000)) continue;
+        const float f = ex2_approx(mw - M);
+        o = __fmaf_rn(f, sm_o[w][g][d], o);
+        L = __fmaf_rn(f, sm_ml[w][g][1], L);
+      }
+    }
+    float* ws = a.workspace + ((int64_t(split) * a.batch + b) * a.heads + h) * int64_t(a.lq) * (D + 2) +
+                int64_t(row) * (D + 2);
+    ws[d] = o;
+    if (d == 0) {
+      ws[D] = M;
+      ws[D + 1] = L;
+    }
+  }
+}
+
 namespace {
 
-// Query rows per CTA (more rows run as more row groups over the same range).
+// Query rows per CTA of the arithmetic form (more rows run as more row groups
+// over the same range).
 constexpr int kDecQG = 1;
+
+// Query rows per CTA: the table form takes two rows together, four with
+// 4-bit codes (the row's partial sums, rows x codes per word, stay <= 32).
+int decode_rows_per_cta(int bits, int lq) {
+  if (bits > 4 || lq <= 1) return 1;
+  return bits == 4 && lq > 2 ? 4 : 2;
+}
 
 template <int BITS, int D, int QG>
 cudaError_t launch_dec(const AttnArgs& a, cudaStream_t stream) {
@@ -796,8 +1128,15 @@ cudaError_t launch_dec(const AttnArgs& a, cudaStream_t stream) {
 
 template <int BITS, int D>
 cudaError_t launch_dec_lut(const AttnArgs& a, cudaStream_t stream) {
-  const dim3 grid(unsigned(a.lq * a.n_splits), unsigned(a.heads), unsigned(a.batch));
-  attn_decode_lut_kernel<BITS, D><<<grid, kDecThreads, 0, stream>>>(a);
+  const int qg = decode_rows_per_cta(BITS, a.lq);
+  const dim3 grid(unsigned((a.lq + qg - 1) / qg * a.n_splits), unsigned(a.heads), unsigned(a.batch));
+  if (qg == 1) {
+    attn_decode_lut_kernel<BITS, D><<<grid, kDecThreads, 0, stream>>>(a);
+  } else if (qg == 2) {
+    attn_decode_lut_rows_kernel<BITS, D, 2><<<grid, kDecThreads, 0, stream>>>(a);
+  } else {
+    if constexpr (BITS == 4) attn_decode_lut_rows_kernel<BITS, D, 4><<<grid, kDecThreads, 0, stream>>>(a);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention_combine(a, stream);
@@ -819,14 +1158,15 @@ cudaError_t launch_dec_bits(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool use_decode_kernel(const AttnArgs& a) {
-  return a.kv_split && !has_rope(a) && a.lq <= kDecodeMaxLq;
+  return a.kv_split && !has_rope(a) && a.lq <= (a.bits <= 4 ? kDecodeTableMaxLq : kDecodeMaxLq);
 }
 
 // About six CTAs per SM over the grid, each warp at least four steps long;
 // then, up to twice that many ranges, the count that fills the last wave of
 // 148 SMs x 2 resident CTAs (128 registers a thread) best.
 int split_kv_decode_splits(const AttnArgs& a) {
-  const int nrg = (a.lq + kDecQG - 1) / kDecQG;
+  const int qg = decode_rows_per_cta(a.bits, a.lq);
+  const int nrg = (a.lq + qg - 1) / qg;
   const int cpw = 32 / a.bits;
   const int rpw = 32 / (a.head_dim / 16);
   const int words = (a.t_att + cpw - 1) / cpw;

@@ -201,9 +201,11 @@ size_t split_kv_workspace_bytes(int batch, int heads, int lq, int head_dim, int 
 // The log-sum-exp merge of the split-KV partials into out (and lse).
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t stream);
 // Split-KV form on the CUDA cores straight from the packed codes (no
-// dequantized tile), for short query blocks without pre-RoPE keys; writes the
-// same partials and runs the same merge.
+// dequantized tile), for short query blocks without pre-RoPE keys: up to two
+// rows (5-8-bit codes), up to four (2-4-bit codes, per-block value tables);
+// writes the same partials and runs the same merge.
 constexpr int kDecodeMaxLq = 2;
+constexpr int kDecodeTableMaxLq = 4;
 bool use_decode_kernel(const AttnArgs& a);
 int split_kv_decode_splits(const AttnArgs& a);
 cudaError_t launch_attention_decode(const AttnArgs& a, cudaStream_t stream);

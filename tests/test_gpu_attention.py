@@ -198,11 +198,13 @@ def test_attention_pre_rope_beyond_fp16_range(bits, path, lq, D):
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("lq", [1, 2])
+@pytest.mark.parametrize("lq", [1, 2, 3, 4])
 def test_attention_decode_from_codes(bits, D, lq):
-    """Split-KV form for one or two query rows (the CUDA-core kernel on the
-    packed codes): block boundaries inside packed words, blocks shorter than a
-    word, a ragged end, several KV ranges per head."""
+    """Split-KV form for one to four query rows (the CUDA-core kernels on the
+    packed codes: one row, or two and four rows per CTA with 2-4-bit codes;
+    5-8-bit codes with three or four rows take the tensor-core split form):
+    block boundaries inside packed words, blocks shorter than a word, a ragged
+    end, several KV ranges per head."""
     B, H = 2, 3
     sizes = [1, 3, 50, 7, 300, 33, 2, 611]
     bs = synth.block_starts(sizes)
@@ -219,14 +221,14 @@ def test_attention_decode_from_codes(bits, D, lq):
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("D", [64, 128])
 def test_attention_decode_block_tables(bits, D):
-    """Split-KV form for one and two query rows with 2-4-bit codes, which the
-    kernel dequantizes through per-block value tables: blocks of 33-700 tokens,
-    so the tables are rebuilt as each KV range moves on and its waves of
-    steps reach one, two or three blocks."""
+    """Split-KV form for one to four query rows with 2-4-bit codes, which the
+    kernels dequantize through per-block value tables: blocks of 33-700
+    tokens, so the tables are rebuilt as each KV range moves on and its waves
+    of steps reach one, two or three blocks."""
     B, H = 1, 3
     sizes = [700, 90, 130, 257, 64, 129, 33, 520, 300]
     bs = synth.block_starts(sizes)
-    for lq in (1, 2):
+    for lq in (1, 2, 3, 4):
         k, v, q, _, _ = _inputs(B, H, D, sizes, lq, seed=bits * 7 + D + lq)
         L = V.varq_cache_alloc(B, H, D, bits, bs)
         out, lse = _gpu_attention(L, k, v, q, len(sizes), path=V.PATH_SPLIT)
@@ -297,8 +299,8 @@ def _sample_rows(lq, rng, n):
 
 FULL = [("var_d16", 4, 256, None), ("infinity_8b", 2, 4096, None), ("infinity_8b", 4, 4096, None),
         ("self_forcing", 4, 4680, None), ("longlive", 2, 4680, None), ("longlive", 3, 4680, None),
-        ("longlive", 4, 4680, None), ("sweep", 4, 1, None), ("sweep", 4, 16, None), ("sweep", 4, 1024, None),
-        ("sweep", 2, 4, None), ("sweep", 8, 64, None)]
+        ("longlive", 4, 4680, None), ("sweep", 4, 1, None), ("sweep", 4, 4, None), ("sweep", 4, 16, None),
+        ("sweep", 4, 1024, None), ("sweep", 2, 4, None), ("sweep", 8, 64, None)]
 
 
 @pytest.mark.parametrize("name,bits,lq,_", FULL, ids=lambda x: str(x))

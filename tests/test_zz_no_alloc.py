@@ -4,7 +4,7 @@ varq_packed_attention_noalloc serves callers that cannot call cudaMalloc
 (their allocator already owns the device memory, or they cannot afford the
 implicit synchronisation): its split partials live in a fixed scratch array
 inside the library.  Calls in a row, of every kernel it can pick (the
-CUDA-core kernel for one or two query rows, the tensor-core split kernel for
+CUDA-core kernels for up to four query rows, the tensor-core split kernel for
 more rows or pre-RoPE keys, and the tensor-core kernel as the fallback when the
 CUDA-core kernel's partials would not fit the array), must each match
 varq_packed_attention's split-KV output and the fp64 oracle within the
@@ -64,8 +64,8 @@ def _agree(ref, ref_lse, out, lse):
 
 
 def test_noalloc_calls_in_a_row_match_the_workspace_entry_point_and_the_oracle():
-    """Five calls in a row on one cache: 16 and 5 query rows (tensor-core split
-    kernel), 1 and 2 rows (CUDA-core kernel), 8 rows with pre-RoPE keys
+    """Six calls in a row on one cache: 16 and 5 query rows (tensor-core split
+    kernel), 1, 2 and 4 rows (CUDA-core kernels), 8 rows with pre-RoPE keys
     (tensor-core split kernel, fp16 scores)."""
     B, H, D, bits = 2, 4, 128, 4
     sizes = [1, 4, 16, 36, 64, 144, 256, 700]
@@ -75,7 +75,7 @@ def test_noalloc_calls_in_a_row_match_the_workspace_entry_point_and_the_oracle()
     kp, km, vp, vm = _cache(L, k.to(DEV), v.to(DEV))
     g = torch.Generator()
     g.manual_seed(4)
-    for call, (lq, rope) in enumerate(((16, False), (5, False), (1, False), (2, False), (8, True))):
+    for call, (lq, rope) in enumerate(((16, False), (5, False), (1, False), (2, False), (4, False), (8, True))):
         q = synth.queries(g, B, H, lq, D)
         c, s = (cos.to(DEV), sin.to(DEV)) if rope else (None, None)
         ref, ref_lse, out, lse = _both(L, q.to(DEV), kp, km, vp, vm, c, s)
