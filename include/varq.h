@@ -213,8 +213,9 @@ VARQ_API size_t varq_packed_attention_workspace(const varq_cache_layout* layout,
  *   path         VARQ_PATH_AUTO (SPLIT for lq <= VARQ_SPLIT_MAX_LQ, else
  *                TENSOR), VARQ_PATH_TENSOR or VARQ_PATH_SPLIT.  SPLIT divides
  *                the cache axis over CTAs and merges their partials; with
- *                lq <= 2 and no rope tables it runs on the CUDA cores straight
- *                from the packed words, otherwise on the tensor cores.
+ *                lq <= 2 (lq <= 4 for 2-4-bit caches) and no rope tables it
+ *                runs on the CUDA cores straight from the packed words,
+ *                otherwise on the tensor cores.
  *                Results agree within the attention tolerance either way.
  *   dev_status   device uint32 or NULL (VARQ_DEV_TIMEOUT).
  */
@@ -291,8 +292,9 @@ VARQ_API int varq_packed_attention_rope3d(const varq_cache_layout* layout,
  *   - Every call shares the one array: calls whose GPU work overlaps (other
  *     streams, other threads) race.  Serialise them.
  *   - The kernel is chosen as in varq_packed_attention: the CUDA-core kernel
- *     for lq <= 2 without rope tables, if its partials fit the array, else the
- *     tensor-core split kernel (fewer ranges, smaller partials).  A shape
+ *     for lq <= 2 (lq <= 4 for 2-4-bit caches) without rope tables, if its
+ *     partials fit the array, else the tensor-core split kernel (fewer
+ *     ranges, smaller partials).  A shape
  *     whose partials fit neither returns VARQ_ERR_WORKSPACE before anything is
  *     launched.  varq_packed_attention_workspace(..., VARQ_PATH_SPLIT) is an
  *     upper bound of what this call needs: a shape whose query is at most

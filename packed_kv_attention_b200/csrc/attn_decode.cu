@@ -4,17 +4,23 @@
 // retrieval": values dequantized to BF16; "Next-block prediction": every query
 // attends to the whole cache).
 //
-// With one or two query rows the tensor-core kernel pads each MMA from 1 row
+// With a few query rows the tensor-core kernel pads each MMA from a few rows
 // to 128 and is bound by writing a 16-bit tile to shared memory.  Here every
-// code is dequantized in registers to the value the definition gives,
-// bf16(fmaf(code, scale, min)), and used at once: K codes in a dot product
-// with the query (pre-scaled by softmax scale x log2 e), V codes in O += P V.
-// A code costs a logic op (OR-ed in place into the mantissa of 2^23), three
-// FMA-pipe ops (exact convert, dequant fma, dot-product fma) and half a bf16
-// pack with its unpack; the ALU pipe is the bound.
+// code is dequantized to the value the definition gives, bf16(fmaf(code,
+// scale, min)), and used at once: K codes in a dot product with the query
+// (pre-scaled by softmax scale x log2 e), V codes in O += P V.  Two forms:
+// - arithmetic (attn_decode_kernel, 5-8-bit codes, one or two rows): a code
+//   costs a logic op (OR-ed in place into the mantissa of 2^23), three
+//   FMA-pipe ops (exact convert, dequant fma, dot-product fma) and half a bf16
+//   pack with its unpack; the ALU pipe is the bound;
+// - tables (attn_decode_lut_kernel for one row, attn_decode_lut_rows_kernel
+//   for two or four rows per CTA, 2-4-bit codes, one to four rows): the 2^b
+//   values of every (block, channel) cell are tabulated in shared memory and
+//   a code costs a byte permute and a shared load (further below).
 //
-// Work split: CTA (KV range, query row, head, batch); its 8 warps take steps
-// of RPW word rows in turn.  K: lane (word row, 16-channel group) forms the
+// Work split (both forms): CTA (KV range, query rows, head, batch); its 8
+// warps take steps of RPW word rows in turn.  K: lane (word row, 16-channel
+// group) forms the
 // partial scores of the row's tokens over its channels, and a reduce-scatter
 // over the row's lanes leaves each lane whole scores.  Each warp keeps its own
 // online-softmax state (running max m, lane-partial sums l, O for the lane's
