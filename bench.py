@@ -370,7 +370,7 @@ def measure_rows(dev, stream, peaks, iters=5):
     workload made for it and against its own roofline:
       a2-a5 quantize+pack and a6 unpack+dequant on the 1 GiB kernel-sweep
             cache (bits 2, 3, 4, 8; inputs and outputs exceed L2);
-      a9    split-KV attention (Lq = 1 and 16) over the sweep cache (INT4);
+      a9    split-KV attention (Lq = 1, 4 and 16) over the sweep cache (INT4);
       a8    pre-RoPE keys: tensor-path attention of the Self-Forcing-like
             next-frame layer (INT4, 4680 queries over 32,760 tokens)."""
     from packed_kv_attention_b200 import varq as V
