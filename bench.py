@@ -821,10 +821,12 @@ def profile_case(name):
         torch.cuda.synchronize()
         for _ in range(3):
             V.varq_unpack_dequant(L, kp, km, out)
-    elif name == "attn_decode_sweep_int4_lq1":
-        # CUDA-core split-KV decode: a quarter of the sweep cache (B2 H32 T16384 D128), INT4, Lq 1
+    elif name in ("attn_decode_sweep_int4_lq1", "attn_decode_sweep_int4_lq4"):
+        # CUDA-core split-KV decode (one row, or four rows per CTA): a quarter of the
+        # sweep cache (B2 H32 T16384 D128), INT4, Lq 1 or 4
+        lq = int(name[-1])
         w = synth.WORKLOADS["sweep"]
-        data = synth.make_inputs(w, lq=1, seed=3, device=dev, batch=2)
+        data = synth.make_inputs(w, lq=lq, seed=3, device=dev, batch=2)
         L = V.varq_cache_alloc(2, w.heads, w.head_dim, 4, data["block_start"])
         kp, km = V.alloc_cache(L, dev)
         vp, vm = V.alloc_cache(L, dev)
@@ -832,7 +834,7 @@ def profile_case(name):
         V.varq_quantize_pack(L, data["v"], vp, vm)
         q = data["q"].contiguous()
         o = torch.empty_like(q)
-        ws = torch.empty(max(V.varq_packed_attention_workspace(L, 1, w.n_blocks) // 4, 1), dtype=torch.float32,
+        ws = torch.empty(max(V.varq_packed_attention_workspace(L, lq, w.n_blocks) // 4, 1), dtype=torch.float32,
                          device=dev)
         torch.cuda.synchronize()
         for _ in range(3):
@@ -844,7 +846,7 @@ def profile_case(name):
 
 
 PROFILE_CASES = ("attn_sk_sweep_int4_lq16", "quant_pack_sweep_b1_int4", "attn_tc2_self_forcing_b2_schedule",
-                 "unpack_dequant_sweep_b1_int4", "attn_decode_sweep_int4_lq1")
+                 "unpack_dequant_sweep_b1_int4", "attn_decode_sweep_int4_lq1", "attn_decode_sweep_int4_lq4")
 
 
 def main(argv=None):
