@@ -444,9 +444,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(const __gri
 // block boundary, or inside a block neither slot holds (waves spanning more
 // than two blocks), takes the per-token path of the kernel above.
 // K channel map: word i of lane (row r, group cg) holds channel
-// cg + NCG m with m = (i & 8) | ((i + r) & 7) (plus 64 (i >> 3) for D = 128),
-// so in every load the 32 lanes read 32 distinct banks; V lanes own channels
-// lane + 32 k as above, one bank each.
+// cg + NCG m with m = (i & 8) | ((i + r) & 7), so in every load the 32 lanes
+// read 32 distinct banks; V lanes own channels lane + 32 k as above, one bank
+// each.
 namespace {
 
 template <int BITS, int D>
