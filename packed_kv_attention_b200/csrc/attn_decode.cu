@@ -1140,8 +1140,10 @@ cudaError_t launch_dec_lut(const AttnArgs& a, cudaStream_t stream) {
     attn_decode_lut_kernel<BITS, D><<<grid, kDecThreads, 0, stream>>>(a);
   } else if (qg == 2) {
     attn_decode_lut_rows_kernel<BITS, D, 2><<<grid, kDecThreads, 0, stream>>>(a);
+  } else if constexpr (BITS == 4) {
+    attn_decode_lut_rows_kernel<BITS, D, 4><<<grid, kDecThreads, 0, stream>>>(a);
   } else {
-    if constexpr (BITS == 4) attn_decode_lut_rows_kernel<BITS, D, 4><<<grid, kDecThreads, 0, stream>>>(a);
+    return cudaErrorInvalidValue;  // four rows per CTA only with 4-bit codes
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
